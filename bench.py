@@ -1,0 +1,494 @@
+"""Benchmark of the DSA hot path on B200: tokens/s at 128K context.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
+
+One JSON line on rank 0.  The headline `value` is prefill tokens/s of the
+128K-token causal prefill (B=1, L=131072, k=2048, indexer 64x128 FP8, 128
+heads over a 576/512 MLA row, score tiles of 4096 query rows).  One step is
+one pass of that prefill through the three steps (indexer -> top-k per query
+block, then sparse attention).  The `decode` object reports the 128K decode
+(B=8 sequences, one query each) the same way, which adds the split-k combine.
+
+Kernel timing: each step calls the C-ABI step entry points in the order
+dsa_forward uses, with CUDA events between launches on the launching stream,
+so every kernel's share of the step is measured live; `e2e` runs dsa_forward
+itself on host (pinned) buffers with the copies inside the timed region.
+
+Inputs are synthetic (long_context_05_b200.inputs), larger than L2 for the
+prefill; L2 is flushed between timed steps anyway (a 256 MiB write outside
+the timed events).  Multi-GPU: one process per GPU, each rank runs its own
+independent sequence(s) (weak scaling, no collective on the data path); the
+step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_05_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "DSA tokens/s (prefill, decode) at 128K ctx; % of HBM / tensor-core roofline"
+PREFILL = "prefill_128k"
+DECODE = "decode_128k_b8"
+FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class Flusher:
+    """Writes a buffer larger than the 126 MB L2 between timed steps."""
+
+    def __init__(self):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+# ------------------------------------------------------------------ work model
+
+def causal_pairs(wl):
+    """(indexer pairs, attention pairs) of one batch: sum over queries of
+    pos + 1 and min(pos + 1, k)."""
+    ip = ap = 0
+    for t in range(wl.T):
+        v = wl.S - wl.T + t + 1
+        ip += v
+        ap += min(v, wl.k)
+    return ip * wl.B, ap * wl.B
+
+
+# ------------------------------------------------------------------ GPU arm
+
+class DsaRunner:
+    """Runs one workload through the C ABI, step by step, with events."""
+
+    def __init__(self, wl, seed_offset=0):
+        from long_context_05_b200 import dsa
+        self.dsa = dsa
+        self.wl = wl = wl.with_(seed=wl.seed + seed_offset)
+        self.inp = make_inputs(wl, "cuda")
+        self.inp.pop("needle_pos", None)
+        self.shape = dsa.make_shape(wl)
+        self.ws = dsa.alloc_workspace(self.shape)
+        self.outs = dsa.alloc_outputs(wl)
+        self.ld = (wl.S + 63) // 64 * 64
+        self.scores = self.ws[: wl.B * self.rows_per_block() * self.ld * 4].view(torch.float32).view(-1, self.ld)
+        self.stream = torch.cuda.current_stream()
+
+    def rows_per_block(self):
+        wl = self.wl
+        return wl.T if wl.decode else min(wl.q_block, wl.T)
+
+    def step(self, ev=None):
+        """One pass of the path via the step entry points; if ev is a list,
+        append (name, start_event, end_event) per launch group."""
+        d, wl, i, o = self.dsa, self.wl, self.inp, self.outs
+        qb = self.rows_per_block()
+
+        def mark():
+            if ev is None:
+                return None
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(self.stream)
+            return e
+
+        for q0 in range(0, wl.T, qb):
+            cnt = min(qb, wl.T - q0)
+            e0 = mark()
+            d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, self.scores)
+            e1 = mark()
+            d.topk(self.shape, self.scores, q0, cnt, o.idx)
+            e2 = mark()
+            if ev is not None:
+                ev.append(("indexer", e0, e1))
+                ev.append(("topk", e1, e2))
+        e3 = mark()
+        d.sparse_attn(self.shape, i["q"], i["kv"], o.idx, o.out, o.lse, self.ws)
+        e4 = mark()
+        if ev is not None:
+            ev.append(("sparse_attn", e3, e4))
+
+    def forward(self):
+        self.dsa.forward(self.shape, self.inp, self.outs.out, self.outs.lse, self.outs.idx, self.ws)
+
+
+def time_steps(runner, steps, warmup, ws):
+    flush = Flusher()
+    for _ in range(warmup):
+        runner.step()
+    torch.cuda.synchronize()
+    st, det = runner.dsa.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {det:#x}")
+    per_kernel = {}
+    total_ms = 0.0
+    launches0 = runner.dsa.launch_count()
+    barrier(ws)
+    torch.cuda.synchronize()
+    for _ in range(steps):
+        flush()
+        ev = []
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record()
+        runner.step(ev)
+        s1.record()
+        s1.synchronize()
+        total_ms += s0.elapsed_time(s1)
+        for name, a, b in ev:
+            per_kernel.setdefault(name, []).append(a.elapsed_time(b))
+    torch.cuda.synchronize()
+    barrier(ws)
+    launches = runner.dsa.launch_count() - launches0
+    st, det = runner.dsa.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {det:#x}")
+    return total_ms, per_kernel, launches
+
+
+def kernel_report(wl, per_kernel, steps, peaks, peak_src, sustained):
+    ip, ap = causal_pairs(wl)
+    bf16 = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    kind = "sustained" if sustained else "burst"
+    work = {
+        # name: (algorithmic amount per step, unit, bound, peak, peak note)
+        "indexer": (2.0 * wl.H_I * wl.D_I * ip / 1e12, "TFLOP/s", "tensor", bf16 * FP8_PER_BF16,
+                    f"fp8 = {kind} bf16 x {FP8_PER_BF16:g} ({peak_src})"),
+        "topk": (4.0 * ip / 1e9, "GB/s", "hbm", peaks["hbm_gbs"], f"hbm ({peak_src})"),
+        "sparse_attn": ((2.0 * wl.H * (wl.d_k + wl.d_v) * ap / 1e12, "TFLOP/s", "tensor", bf16,
+                         f"bf16 {kind} ({peak_src})") if not wl.decode else
+                        (2.0 * wl.d_k * ap / 1e9, "GB/s", "hbm", peaks["hbm_gbs"], f"hbm, gathered KV bytes ({peak_src})")),
+    }
+    out = {}
+    tot = sum(sum(v) for v in per_kernel.values())
+    for name, times in per_kernel.items():
+        ms = sum(times) / steps                       # per step
+        launches = len(times) / steps
+        amount, unit, bound, peak, note = work[name]
+        achieved = amount / (ms / 1e3)
+        out[name] = {"ms_per_step": ms, "launches_per_step": launches, "share": sum(times) / tot,
+                     "bound": bound, "achieved": achieved, "unit": unit, "peak": peak,
+                     "frac": achieved / peak, "peak_note": note,
+                     "work_per_step": amount * (1e12 if unit == "TFLOP/s" else 1e9)}
+    return out
+
+
+def cpu_oracle_sample(wl, inp, budget_s=12.0, max_rows=64):
+    """The FP64 oracle as it stands, on evenly spread query rows of the same
+    workload (one full path per row), until the time budget is used."""
+    import numpy as np
+    from oracle import dsa_oracle as O
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    b = 0
+    kd = O.e4m3_decode(inp["k_I"][b].cpu().numpy()) * inp["k_scale"][b].cpu().double().numpy()[:, None]
+    kv = O.bf16_decode(u16(inp["kv"][b]))
+    tau = O.default_tau(wl.d_k)
+    n_target = max_rows
+    rows = [int(wl.T * (i + 0.5) / n_target) for i in range(n_target)]
+    rng = np.random.default_rng(0)
+    rng.shuffle(rows)
+    done = 0
+    t0 = time.perf_counter()
+    for t in rows:
+        qd = O.e4m3_decode(inp["q_I"][b, t].cpu().numpy()) * inp["q_scale"][b, t].cpu().double().numpy()[:, None]
+        w = inp["w"][b, t].cpu().double().numpy()
+        q = O.bf16_decode(u16(inp["q"][b, t]))
+        O.dsa_row(qd, w, kd, q, kv, O.query_pos(wl.T, wl.S, t), wl.k, wl.d_v, tau)
+        done += 1
+        if time.perf_counter() - t0 > budget_s and done >= 4:
+            break
+    el = time.perf_counter() - t0
+    try:
+        import threadpoolctl
+        cores = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) or 1
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": done / el * wl.B, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} query rows of {wl.name} spread evenly over positions 0..{wl.T - 1}, "
+                      f"full path per row (indexer over pos+1 keys, top-k, attention), {el:.1f} s"}
+
+
+def run_e2e(runner, steps, ws):
+    """dsa_forward on pinned host buffers: H2D of the inputs, the call, D2H of
+    out and lse, all inside the timed region."""
+    wl = runner.wl
+    host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in runner.inp.items()}
+    for k, v in runner.inp.items():
+        host_in[k].copy_(v)
+    host_out = torch.empty(runner.outs.out.shape, dtype=torch.bfloat16, pin_memory=True)
+    host_lse = torch.empty(runner.outs.lse.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4
+
+    def one():
+        for k, v in host_in.items():
+            runner.inp[k].copy_(v, non_blocking=True)
+        runner.forward()
+        host_out.copy_(runner.outs.out, non_blocking=True)
+        host_lse.copy_(runner.outs.lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(ws)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(steps):
+        one()
+    s1.record()
+    s1.synchronize()
+    ms = max_over_ranks(s0.elapsed_time(s1) / steps, ws)
+    del host_in
+    return ms, h2d, d2h
+
+
+def gpu_arm(args):
+    ws, rank, local = dist_setup(args.gpus)
+    from long_context_05_b200 import dsa
+    dsa.lib()
+    peaks, peak_src = load_peaks()
+    wl = WORKLOADS[args.workload]
+    wl_dec = WORKLOADS[args.decode_workload] if args.decode_workload != "none" else None
+
+    clocks = ClockSampler(local)
+
+    runner = DsaRunner(wl, seed_offset=rank)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(runner.wl, runner.inp, budget_s=args.cpu_seconds)
+
+    clocks.start()
+    total_ms, per_kernel, launches = time_steps(runner, args.steps, args.warmup, ws)
+    ms_step = max_over_ranks(total_ms / args.steps, ws)
+    dec = None
+    if wl_dec is not None:
+        drun = DsaRunner(wl_dec, seed_offset=rank)
+        d_total, d_kern, d_launch = time_steps(drun, args.steps, args.warmup, ws)
+        d_ms = max_over_ranks(d_total / args.steps, ws)
+        d_rep = kernel_report(drun.wl, d_kern, args.steps, peaks, peak_src, sustained=False)
+        d_top = max(d_rep.items(), key=lambda kv: kv[1]["ms_per_step"])
+        dec = {"workload": wl_dec.name, "value": ws * wl_dec.B * wl_dec.T / (d_ms / 1e3), "unit": "tokens/s",
+               "ms_per_step": d_ms, "gpu_launches": d_launch,
+               "config": {"batch": wl_dec.B, "context": wl_dec.S, "k": wl_dec.k, "H": wl_dec.H,
+                          "H_I": wl_dec.H_I, "D_I": wl_dec.D_I, "d_k": wl_dec.d_k, "d_v": wl_dec.d_v},
+               "roofline": {"kernel": d_top[0], "bound": d_top[1]["bound"], "achieved": d_top[1]["achieved"],
+                            "peak": d_top[1]["peak"], "unit": d_top[1]["unit"], "frac": d_top[1]["frac"],
+                            "traffic": None},
+               "kernels": d_rep}
+        del drun
+    clk = clocks.stop()
+
+    e2e = None
+    need = sum(v.numel() * v.element_size() for v in runner.inp.values()) + runner.outs.out.numel() * 2
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    if not args.no_e2e and avail is not None and avail < 2 * need * max(1, ws):
+        e2e = {"skipped": f"host RAM available {avail / 2**30:.0f} GiB < 2 x {need / 2**30:.0f} GiB pinned per rank"}
+    elif not args.no_e2e:
+        e_ms, h2d, d2h = run_e2e(runner, args.e2e_steps, ws)
+        e2e = {"value": ws * wl.B * wl.T / (e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    rep = kernel_report(runner.wl, per_kernel, args.steps, peaks, peak_src, sustained=True)
+    top = max(rep.items(), key=lambda kv: kv[1]["ms_per_step"])
+    tokens = ws * wl.B * wl.T
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8 indexer (f32 accumulate) / bf16 attention (f32 accumulate)",
+        "data": "synthetic (seeded; needles + local-window bias), inputs larger than L2, L2 flushed between steps",
+        "config": {"workload": wl.name, "batch": wl.B, "seq_len": wl.T, "context": wl.S, "k": wl.k,
+                   "q_block": wl.q_block, "H_I": wl.H_I, "D_I": wl.D_I, "H": wl.H, "d_k": wl.d_k,
+                   "d_v": wl.d_v, "parallelism": f"independent sequences x{ws}", "l2": "flushed between steps"},
+        "gpu_launches": launches // args.steps,
+        "roofline": {"kernel": top[0], "bound": top[1]["bound"], "achieved": top[1]["achieved"],
+                     "peak": top[1]["peak"], "unit": top[1]["unit"], "frac": top[1]["frac"], "traffic": None,
+                     "peak_note": top[1]["peak_note"]},
+        "kernels": rep,
+        "decode": dec,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "peaks_source": peak_src,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def reference_arm(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(wl.with_(T=wl.T, S=wl.S), dev) if dev == "cuda" else None
+    if inp is None:
+        # generate on the host when there is no GPU; same shapes, CPU stream
+        inp = make_inputs(wl, "cpu")
+    vals = []
+    cpu = None
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(wl, inp, budget_s=args.cpu_seconds / max(1, args.steps), max_rows=16)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            cpu = r
+    v = statistics.mean(vals)
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * wl.B * wl.T / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "seq_len": wl.T, "context": wl.S, "k": wl.k},
+            "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cpu["cores"], "kind": "oracle",
+                             "sample": cpu["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--workload", default=PREFILL, choices=sorted(WORKLOADS))
+    ap.add_argument("--decode-workload", default=DECODE, choices=sorted(WORKLOADS) + ["none"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "dsa":
+        print("note: warm-up raised to the minimum of 3 steps", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,294 @@
+// Host side of libdsa.so: argument checks, workspace layout, launch order.
+// The arithmetic of every step lives in the kernel files; this file only
+// validates, carves the caller's workspace and enqueues launches.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "internal.h"
+
+namespace dsa {
+
+__device__ DevErr g_dsa_err;
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kDefaultSpinLimit = 1LL << 26;  // about 0.1-1 s of polling
+long long g_spin_limit = kDefaultSpinLimit;
+
+struct DeviceInfo {
+  DevErr* err = nullptr;
+  int num_sms = 0;
+  bool ready = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+dsa_status device_info(DeviceInfo* out, int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dsa_err) != cudaSuccess) return DSA_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DSA_ERR_CUDA;
+    d.err = static_cast<DevErr*>(p);
+    d.num_sms = sms;
+    d.ready = true;
+  }
+  *out = d;
+  *dev_out = dev;
+  return DSA_OK;
+}
+
+dsa_status make_ctx(void* stream, LaunchCtx* c) {
+  DeviceInfo d;
+  int dev = 0;
+  dsa_status st = device_info(&d, &dev);
+  if (st != DSA_OK) return st;
+  c->stream = static_cast<cudaStream_t>(stream);
+  c->err = d.err;
+  c->spin_limit = g_spin_limit;
+  c->num_sms = d.num_sms;
+  c->device = dev;
+  return DSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool is_pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// Basic validity of the shape (sizes positive, ranges supported).
+dsa_status check_shape(const dsa_shape* s) {
+  if (s == nullptr) return DSA_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->T <= 0 || s->S <= 0 || s->k <= 0 || s->H <= 0 || s->H_I <= 0 || s->D_I <= 0 ||
+      s->d_k <= 0 || s->d_v <= 0)
+    return DSA_ERR_INVALID_ARG;
+  if (s->T > s->S) return DSA_ERR_INVALID_ARG;
+  if (s->mode != DSA_PREFILL && s->mode != DSA_DECODE) return DSA_ERR_INVALID_ARG;
+  if (s->D_I != 32 && s->D_I != 64 && s->D_I != 128) return DSA_ERR_UNSUPPORTED;
+  if (!is_pow2_in(s->H_I, 4, 64)) return DSA_ERR_UNSUPPORTED;
+  if (!((s->d_k == 576 && s->d_v == 512) || (s->d_k == 80 && s->d_v == 64))) return DSA_ERR_UNSUPPORTED;
+  if (s->H > 128 || s->H % 8 != 0) return DSA_ERR_UNSUPPORTED;
+  if (s->k > 2048) return DSA_ERR_UNSUPPORTED;
+  if ((long long)s->S >= (1LL << 31) / 8) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+int q_block_of(const dsa_shape* s) {
+  int qb = s->q_block > 0 ? s->q_block : 4096;
+  return qb < s->T ? qb : s->T;
+}
+
+int64_t scores_ld(const dsa_shape* s) { return (int64_t)round_up((size_t)s->S, 64); }
+
+float tau_of(const dsa_shape* s) {
+  return s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / sqrtf((float)s->d_k);
+}
+
+// Workspace layout (each region 256-byte aligned):
+//   [scores: B * q_rows * ld floats][attention split partials]
+struct WsLayout {
+  size_t scores_off, scores_bytes;
+  size_t part_off, part_bytes;
+  size_t total;
+  int nsplit;
+  int q_rows;
+};
+
+WsLayout ws_layout(const dsa_shape* s, int num_sms) {
+  WsLayout L;
+  L.q_rows = s->mode == DSA_DECODE ? s->T : q_block_of(s);
+  L.scores_off = 0;
+  L.scores_bytes = round_up((size_t)s->B * L.q_rows * scores_ld(s) * sizeof(float), 256);
+  L.nsplit = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->k, num_sms) : 1;
+  L.part_off = L.scores_off + L.scores_bytes;
+  L.part_bytes = round_up(attn_partial_floats(s->B * s->T, s->H, s->d_v, L.nsplit) * sizeof(float), 256);
+  L.total = L.part_off + L.part_bytes;
+  return L;
+}
+
+dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+dsa_status run_indexer(const LaunchCtx& c, const dsa_shape* s, const uint8_t* q_I, const float* q_scale,
+                       const float* w, const uint8_t* k_I, const float* k_scale, int q_begin, int q_count,
+                       float* scores, int64_t ld) {
+  IndexerArgs a;
+  a.q_I = q_I; a.q_scale = q_scale; a.w = w; a.k_I = k_I; a.k_scale = k_scale;
+  a.scores = scores; a.ld = ld;
+  a.B = s->B; a.T = s->T; a.S = s->S; a.H_I = s->H_I; a.D_I = s->D_I;
+  a.q_begin = q_begin; a.q_count = q_count;
+  return from_cuda(launch_indexer(c, a));
+}
+
+dsa_status run_topk(const LaunchCtx& c, const dsa_shape* s, const float* scores, int64_t ld, int q_begin,
+                    int q_count, int32_t* idx) {
+  TopkArgs a;
+  a.scores = scores; a.ld = ld; a.idx = idx;
+  a.B = s->B; a.T = s->T; a.S = s->S; a.k = s->k;
+  a.q_begin = q_begin; a.q_count = q_count;
+  return from_cuda(launch_topk(c, a));
+}
+
+dsa_status run_attn(const LaunchCtx& c, const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
+                    const int32_t* idx, uint16_t* out, float* lse, float* part, int nsplit) {
+  AttnArgs a;
+  a.q = q; a.kv = kv; a.idx = idx; a.out = out; a.lse = lse; a.part = part;
+  a.B = s->B; a.T = s->T; a.S = s->S; a.H = s->H; a.d_k = s->d_k; a.d_v = s->d_v; a.k = s->k;
+  a.nsplit = nsplit;
+  a.tau = tau_of(s);
+  return from_cuda(launch_sparse_attn(c, a));
+}
+
+bool indexer_ptrs_ok(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_I,
+                     const float* k_scale) {
+  return q_I && q_scale && w && k_I && k_scale && aligned16(q_I) && aligned16(k_I);
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+const char* dsa_status_string(dsa_status st) {
+  switch (st) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_DEVICE_BOUNDS: return "device index out of bounds";
+  }
+  return "unknown status";
+}
+
+unsigned long long dsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void dsa_set_spin_limit(long long iterations) {
+  g_spin_limit = iterations > 0 ? iterations : kDefaultSpinLimit;
+}
+
+size_t dsa_workspace_size(const dsa_shape* s) {
+  if (check_shape(s) != DSA_OK) return 0;
+  DeviceInfo d;
+  int dev = 0;
+  int sms = 148;
+  if (device_info(&d, &dev) == DSA_OK) sms = d.num_sms;
+  return ws_layout(s, sms).total;
+}
+
+dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_I, const float* q_scale, const float* w,
+                              const uint8_t* k_I, const float* k_scale, int q_begin, int q_count,
+                              float* scores, int64_t ld_scores, void* stream) {
+  dsa_status st = check_shape(s);
+  if (st != DSA_OK) return st;
+  if (!indexer_ptrs_ok(q_I, q_scale, w, k_I, k_scale) || scores == nullptr || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > s->T) return DSA_ERR_INVALID_ARG;
+  if (ld_scores < s->S || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
+  return run_indexer(c, s, q_I, q_scale, w, k_I, k_scale, q_begin, q_count, scores, ld_scores);
+}
+
+dsa_status dsa_topk(const dsa_shape* s, const float* scores, int64_t ld_scores, int q_begin, int q_count,
+                    int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws; (void)ws_bytes;
+  dsa_status st = check_shape(s);
+  if (st != DSA_OK) return st;
+  if (scores == nullptr || idx == nullptr) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > s->T) return DSA_ERR_INVALID_ARG;
+  if (ld_scores < s->S) return DSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
+  return run_topk(c, s, scores, ld_scores, q_begin, q_count, idx);
+}
+
+dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                           uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  dsa_status st = check_shape(s);
+  if (st != DSA_OK) return st;
+  if (!q || !kv || !idx || !out || !aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
+  WsLayout L = ws_layout(s, c.num_sms);
+  float* part = nullptr;
+  if (L.part_bytes > 0) {
+    if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.part_off);
+  }
+  return run_attn(c, s, q, kv, idx, out, lse, part, L.nsplit);
+}
+
+dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, float* lse, int32_t* idx_out,
+                       void* ws, size_t ws_bytes, void* stream) {
+  dsa_status st = check_shape(s);
+  if (st != DSA_OK) return st;
+  if (in == nullptr || out == nullptr || idx_out == nullptr) return DSA_ERR_INVALID_ARG;
+  if (!indexer_ptrs_ok(in->q_I, in->q_scale, in->w, in->k_I, in->k_scale)) return DSA_ERR_INVALID_ARG;
+  if (!in->q || !in->kv || !aligned16(in->q) || !aligned16(in->kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
+  WsLayout L = ws_layout(s, c.num_sms);
+  if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + L.scores_off);
+  float* part = L.part_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) + L.part_off) : nullptr;
+  const int64_t ld = scores_ld(s);
+  for (int q0 = 0; q0 < s->T; q0 += L.q_rows) {
+    const int cnt = (s->T - q0) < L.q_rows ? (s->T - q0) : L.q_rows;
+    if ((st = run_indexer(c, s, in->q_I, in->q_scale, in->w, in->k_I, in->k_scale, q0, cnt, scores, ld)) != DSA_OK)
+      return st;
+    if ((st = run_topk(c, s, scores, ld, q0, cnt, idx_out)) != DSA_OK) return st;
+  }
+  return run_attn(c, s, in->q, in->kv, idx_out, out, lse, part, L.nsplit);
+}
+
+dsa_status dsa_prefill(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, float* lse, int32_t* idx_out,
+                       void* ws, size_t ws_bytes, void* stream) {
+  if (s == nullptr) return DSA_ERR_INVALID_ARG;
+  dsa_shape m = *s;
+  m.mode = DSA_PREFILL;
+  return dsa_forward(&m, in, out, lse, idx_out, ws, ws_bytes, stream);
+}
+
+dsa_status dsa_decode(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, float* lse, int32_t* idx_out,
+                      void* ws, size_t ws_bytes, void* stream) {
+  if (s == nullptr) return DSA_ERR_INVALID_ARG;
+  if (s->T != 1) return DSA_ERR_INVALID_ARG;
+  dsa_shape m = *s;
+  m.mode = DSA_DECODE;
+  return dsa_forward(&m, in, out, lse, idx_out, ws, ws_bytes, stream);
+}
+
+dsa_status dsa_get_device_error(void* stream, int* detail) {
+  if (detail) *detail = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  DeviceInfo d;
+  int dev = 0;
+  dsa_status st = device_info(&d, &dev);
+  if (st != DSA_OK) return st;
+  DevErr host = {0u, 0u};
+  if (cudaMemcpy(&host, d.err, sizeof(DevErr), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  DevErr zero = {0u, 0u};
+  if (cudaMemcpy(d.err, &zero, sizeof(DevErr), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
+  if (detail) *detail = (int)host.detail;
+  return static_cast<dsa_status>(host.code);
+}
+
+}  // extern "C"
