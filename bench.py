@@ -279,7 +279,7 @@ def kernel_report(wl, per_kernel, steps, peaks, peak_src, sustained):
     return out
 
 
-def cpu_oracle_sample(wl, inp, budget_s=12.0, max_rows=64):
+def cpu_oracle_sample(wl, inp, budget_s=12.0, max_rows=4096):
     """The FP64 oracle as it stands, on evenly spread query rows of the same
     workload (one full path per row), until the time budget is used."""
     import numpy as np

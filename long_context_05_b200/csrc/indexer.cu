@@ -1,83 +1,415 @@
-// Step A: lightning indexer scores.
+// Step A: lightning indexer scores on the tcgen05 tensor cores (FP8).
 //
 // I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]) over the dequantised FP8
 // operands (ouchyi thread on DeepSeek Sparse Attention, "Nasil calisiyor"
 // paragraph: few heads, FP8, cheap; tenelement.pl, "DeepSeek V3.2-Exp Cuts
 // Long-Context Costs ...", section "Architektura DeepSeek V3.2-Exp: Od MoE do
 // DSA": logits for the context tokens through a ReLU).  Both scales are > 0,
-// so ReLU(a b x) = a b ReLU(x): the kernel folds w * q_scale per query head
-// and k_scale per key after the ReLU and works on the raw e4m3 values.
-#include <cuda_fp8.h>
-
+// so ReLU(a b x) = a b ReLU(x): the MMA runs on the raw e4m3 bytes and the
+// epilogue applies w * q_scale per (query, head) and k_scale per key.
+//
+// Tiling.  One MMA tile is M = 128 keys (A = k_I rows, K-major) by N = 128
+// (query, head) rows of q_I (B, K-major), K = D_I; putting the keys on M makes
+// the sum over the indexer heads a sum along one TMEM lane, i.e. inside one
+// epilogue thread.  A work item is a group of up to 8 such B sub-tiles (16
+// queries at 64 heads) kept in shared memory, times a run of up to 32 key
+// tiles streamed through a 4-stage TMA ring; every key tile feeds all
+// sub-tiles, so each byte of k_I fetched serves 8 MMAs.  Tiles entirely
+// above the causal diagonal are skipped.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over the work items):
+//   warp 0      TMA producer (one elected lane)
+//   warp 1      TMEM allocator and MMA issuer (one elected lane)
+//   warps 2..9  epilogue: two groups of four warps (one per TMEM lane
+//               quarter); group g drains accumulators u with u % 2 == g
+// Four TMEM accumulators of 128 columns each let the MMA run up to three
+// sub-tiles ahead of the epilogue.
 #include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
 
 namespace dsa {
 namespace {
 
-__device__ __forceinline__ float e4m3_to_float(uint8_t b) {
-  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
-  return __half2float(__half(h));
+using namespace sm100;
+
+constexpr int kBM = 128;       // keys per tile (MMA M)
+constexpr int kNSub = 128;     // MMA N: (query, head) rows per sub-tile
+constexpr int kMaxNB = 8;      // sub-tiles per work item
+constexpr int kKC = 32;        // key tiles per work item
+constexpr int kStages = 4;     // depth of the k_I ring
+constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * kNSub = 512 columns)
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;
+
+struct IdxParams {
+  const float* w;
+  const float* q_scale;
+  const float* k_scale;
+  float* scores;
+  long long ld;
+  int B, T, S, q_begin, q_count;
+  int nb;              // B sub-tiles per item
+  int groups_per_seq;  // query groups per sequence
+  long long spin;
+  DevErr* err;
+};
+
+template <int DI>
+struct Layout {
+  static constexpr int kABytes = kBM * DI;
+  static constexpr int kBSubBytes = kNSub * DI;
+  static constexpr int kBOff = 0;
+  static constexpr int kAOff = kBOff + kMaxNB * kBSubBytes;
+  static constexpr int kWOff = kAOff + kStages * kABytes;            // wM, two item buffers
+  static constexpr int kWFloats = kMaxNB * kNSub;
+  static constexpr int kBarOff = kWOff + 2 * kWFloats * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 * kNAcc + 1 + 2;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+  static constexpr uint32_t kSwizzleLayout = DI == 128 ? kSwizzle128 : DI == 64 ? kSwizzle64 : kSwizzle32;
+  static constexpr uint32_t kSBO = 8 * DI;   // 8 rows per swizzle atom
+};
+
+// Work enumeration shared by all roles: items are (sequence, query group,
+// key chunk); CTA `cta` takes every item whose flat index is cta mod grid.
+struct Item {
+  int b, t0, tend, c, ntiles;
+};
+
+template <int HI, class F>
+__device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
+  constexpr int QPS = kNSub / HI;
+  const int per_group = p.nb * QPS;
+  const int grid = gridDim.x, cta = blockIdx.x;
+  long long flat = 0;
+  const int q_end = p.q_begin + p.q_count;
+  for (int gid = 0; gid < p.B * p.groups_per_seq; ++gid) {
+    const int b = gid / p.groups_per_seq;
+    const int g = gid - b * p.groups_per_seq;
+    Item it;
+    it.b = b;
+    it.t0 = p.q_begin + g * per_group;
+    it.tend = min(it.t0 + per_group, q_end);
+    const int pos_last = p.S - p.T + it.tend - 1;
+    it.ntiles = pos_last / kBM + 1;
+    const int nch = (it.ntiles + kKC - 1) / kKC;
+    int c0 = (int)(((long long)cta - flat) % grid);
+    if (c0 < 0) c0 += grid;
+    for (int c = c0; c < nch; c += grid) {
+      it.c = c;
+      if (!f(it)) return;
+    }
+    flat += nch;
+  }
 }
 
-constexpr int kKeysPerBlock = 128;
+// sub-tile j of an item covers queries [t0 + j*QPS, min(t0 + (j+1)*QPS, tend))
+template <int HI>
+__device__ __forceinline__ bool subtile_active(const IdxParams& p, const Item& it, int j, int kt) {
+  constexpr int QPS = kNSub / HI;
+  const int qa = it.t0 + j * QPS;
+  if (qa >= it.tend) return false;
+  const int qlast = min(qa + QPS, it.tend) - 1;
+  return kt * kBM <= p.S - p.T + qlast;
+}
 
-// One block: one query t of sequence b, 128 consecutive keys; one thread per key.
-template <int DI>
-__global__ void __launch_bounds__(kKeysPerBlock) indexer_cuda_core_kernel(IndexerArgs a) {
-  extern __shared__ float smem[];
-  float* qf = smem;                 // [H_I][DI] raw e4m3 values
-  float* wq = smem + a.H_I * DI;    // [H_I] w * q_scale
-  const int b = blockIdx.z;
-  const int i = blockIdx.y;
-  const int t = a.q_begin + i;
-  const int pos = a.S - a.T + t;
-  const int s0 = blockIdx.x * kKeysPerBlock;
-  if (s0 > pos) return;
+__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
 
-  const size_t qrow = (size_t)b * a.T + t;
-  const uint8_t* qp = a.q_I + qrow * a.H_I * DI;
-  for (int x = threadIdx.x; x < a.H_I * DI; x += blockDim.x) qf[x] = e4m3_to_float(qp[x]);
-  for (int j = threadIdx.x; j < a.H_I; j += blockDim.x)
-    wq[j] = a.w[qrow * a.H_I + j] * a.q_scale[qrow * a.H_I + j];
+template <int DI, int HI>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                      IdxParams p) {
+  using L = Layout<DI>;
+  constexpr int QPS = kNSub / HI;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem + L::kBOff;
+  uint8_t* sA = smem + L::kAOff;
+  float* sW = reinterpret_cast<float*>(smem + L::kWOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + kStages;
+  uint64_t* b_full = bars + 2 * kStages;
+  uint64_t* b_empty = b_full + 1;
+  uint64_t* acc_full = b_full + 2;
+  uint64_t* acc_empty = acc_full + kNAcc;
+  uint64_t* mma_done = acc_empty + kNAcc;
+  uint64_t* w_ready = mma_done + 1;  // [2]: epilogue threads finished filling wM buffer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+    }
+    mbar_init(b_full, 1);
+    mbar_init(b_empty, 1);
+    for (int i = 0; i < kNAcc; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);  // one arrive per epilogue warp of the owning group
+    }
+    mbar_init(mma_done, 1);
+    mbar_init(&w_ready[0], kEpiThreads);
+    mbar_init(&w_ready[1], kEpiThreads);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kNAcc * kNSub);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 
-  const int s = s0 + threadIdx.x;
-  if (s > pos) return;
-  const uint8_t* kp = a.k_I + ((size_t)b * a.S + s) * DI;
-  float kf[DI];
+  auto fail = [&](unsigned where) {
+    report_error(p.err, DSA_ERR_TIMEOUT, ERR_SITE_INDEXER | (where << 8));
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_q);
+      uint32_t a_cnt = 0, items = 0;
+      uint32_t last_phase[kStages];
+      bool issued[kStages];
+      for (int i = 0; i < kStages; ++i) issued[i] = false;
+      bool ok = true;
+      for_each_item<HI>(p, [&](const Item& it) {
+        if (!mbar_wait(b_empty, (items & 1) ^ 1, p.spin, abort_flag)) { fail(1); ok = false; return false; }
+        int nsub = 0;
+        for (int j = 0; j < p.nb; ++j)
+          if (it.t0 + j * QPS < it.tend) nsub = j + 1;
+        mbar_arrive_expect_tx(b_full, nsub * L::kBSubBytes);
+        for (int j = 0; j < nsub; ++j)
+          tma_load_2d(sB + j * L::kBSubBytes, &tm_q, b_full, 0, (it.b * p.T + it.t0 + j * QPS) * HI);
+        ++items;
+        const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
+        for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
+          const int st = a_cnt % kStages;
+          if (!mbar_wait(&a_empty[st], ((a_cnt / kStages) & 1) ^ 1, p.spin, abort_flag)) {
+            fail(2); ok = false; return false;
+          }
+          mbar_arrive_expect_tx(&a_full[st], L::kABytes);
+          tma_load_2d(sA + st * L::kABytes, &tm_k, &a_full[st], 0, it.b * p.S + kt * kBM);
+          issued[st] = true;
+          last_phase[st] = (a_cnt / kStages) & 1;
+        }
+        return true;
+      });
+      // let every load this CTA started land before it exits
+      for (int st = 0; st < kStages; ++st)
+        if (issued[st]) mbar_wait(&a_full[st], last_phase[st], p.spin, nullptr);
+      if (items > 0) mbar_wait(b_full, (items - 1) & 1, p.spin, nullptr);
+      (void)ok;
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc(kFmtE4M3, kFmtE4M3, 0, 0, kBM, kNSub);
+      uint32_t a_cnt = 0, items = 0, u = 0;
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      for_each_item<HI>(p, [&](const Item& it) {
+        if (!mbar_wait(b_full, items & 1, p.spin, abort_flag)) { fail(3); return false; }
+        ++items;
+        const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
+        for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
+          const int st = a_cnt % kStages;
+          if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.spin, abort_flag)) { fail(4); return false; }
+          tc_fence_after();
+          const uint64_t adesc = make_sdesc(a_base + st * L::kABytes, 16, L::kSBO, L::kSwizzleLayout);
+          for (int j = 0; j < p.nb; ++j) {
+            if (!subtile_active<HI>(p, it, j, kt)) continue;
+            const int acc = u % kNAcc;
+            if (!mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.spin, abort_flag)) { fail(5); return false; }
+            tc_fence_after();
+            const uint64_t bdesc = make_sdesc(b_base + j * L::kBSubBytes, 16, L::kSBO, L::kSwizzleLayout);
 #pragma unroll
-  for (int d = 0; d < DI; d += 16) {
-    uint4 v = *reinterpret_cast<const uint4*>(kp + d);
-    const uint8_t* vb = reinterpret_cast<const uint8_t*>(&v);
+            for (int ks = 0; ks < DI / 32; ++ks)
+              mma_f8(tmem_base + acc * kNSub, adesc + 2 * ks, bdesc + 2 * ks, idesc, ks > 0 ? 1u : 0u);
+            mma_commit(&acc_full[acc]);
+            ++u;
+          }
+          mma_commit(&a_empty[st]);
+        }
+        mma_commit(b_empty);
+        return true;
+      });
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, p.spin, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int ew = warp - 2;             // 0..7
+    const int grp = ew >> 2;             // accumulator parity this warp drains
+    const int quarter = warp & 3;        // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;   // key row within the tile
+    const int etid = threadIdx.x - 64;   // 0..255
+    uint32_t u = 0, items = 0;
+    for_each_item<HI>(p, [&](const Item& it) {
+      // per-item head weights  wM[(query, head)] = w * q_scale  (0 past the end)
+      float* wbuf = sW + (items & 1) * L::kWFloats;
+      for (int x = etid; x < p.nb * kNSub; x += kEpiThreads) {
+        const int t = it.t0 + x / HI;
+        float v = 0.f;
+        if (t < it.tend) {
+          const size_t o = ((size_t)it.b * p.T + t) * HI + (x % HI);
+          v = p.w[o] * p.q_scale[o];
+        }
+        wbuf[x] = v;
+      }
+      mbar_arrive(&w_ready[items & 1]);
+      if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.spin, abort_flag)) { fail(7); return false; }
+      ++items;
+      const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
+      for (int kt = kt0; kt < kt1; ++kt) {
+        const int s = kt * kBM + r;
+        const float ks = s < p.S ? p.k_scale[(size_t)it.b * p.S + s] : 0.f;
+        for (int j = 0; j < p.nb; ++j) {
+          if (!subtile_active<HI>(p, it, j, kt)) continue;
+          const uint32_t my = u++;
+          if ((int)(my & 1) != grp) continue;
+          const int acc = my % kNAcc;
+          if (!mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.spin, abort_flag)) { fail(6); return false; }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kNSub;
+          const float* wq = wbuf + j * kNSub;
+          float accq[QPS];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) kf[d + e] = e4m3_to_float(vb[e]);
+          for (int q = 0; q < QPS; ++q) accq[q] = 0.f;
+          uint32_t v[2][32];
+          tmem_ld32(taddr, v[0]);
+          tmem_wait_ld_dep(v[0]);
+#pragma unroll
+          for (int c = 0; c < kNSub / 32; ++c) {
+            if (c + 1 < kNSub / 32) {
+              tmem_ld32(taddr + (c + 1) * 32, v[(c + 1) & 1]);
+            } else {
+              // every column of this accumulator is in registers: hand it back
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 w4 = *reinterpret_cast<const float4*>(wq + c * 32 + e);
+              const int q = (c * 32 + e) / HI;
+              float a = accq[q];
+              a = fmaf(w4.x, fmaxf(__uint_as_float(v[c & 1][e + 0]), 0.f), a);
+              a = fmaf(w4.y, fmaxf(__uint_as_float(v[c & 1][e + 1]), 0.f), a);
+              a = fmaf(w4.z, fmaxf(__uint_as_float(v[c & 1][e + 2]), 0.f), a);
+              a = fmaf(w4.w, fmaxf(__uint_as_float(v[c & 1][e + 3]), 0.f), a);
+              accq[q] = a;
+            }
+            if (c + 1 < kNSub / 32) tmem_wait_ld_dep(v[(c + 1) & 1]);
+          }
+#pragma unroll
+          for (int q = 0; q < QPS; ++q) {
+            const int t = it.t0 + j * QPS + q;
+            if (t < it.tend && s <= p.S - p.T + t)
+              p.scores[((size_t)it.b * p.q_count + (t - p.q_begin)) * p.ld + s] = accq[q] * ks;
+          }
+        }
+      }
+      return true;
+    });
   }
-  float acc = 0.f;
-  for (int j = 0; j < a.H_I; ++j) {
-    const float* qj = qf + j * DI;
-    float dot = 0.f;
-#pragma unroll
-    for (int d = 0; d < DI; ++d) dot = fmaf(qj[d], kf[d], dot);
-    acc = fmaf(wq[j], fmaxf(dot, 0.f), acc);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kNAcc * kNSub);
   }
-  a.scores[((size_t)b * a.q_count + i) * a.ld + s] = acc * a.k_scale[(size_t)b * a.S + s];
+}
+
+template <int DI, int HI>
+cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
+  using L = Layout<DI>;
+  constexpr int QPS = kNSub / HI;
+  CUtensorMap tm_k, tm_q;
+  const CUtensorMapSwizzle sw = DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : DI == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                           : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!make_tmap_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.k_I, (uint64_t)a.B * a.S, DI, DI, kBM, DI, sw))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_I, (uint64_t)a.B * a.T * HI, DI, DI, kNSub, DI, sw))
+    return cudaErrorInvalidValue;
+  IdxParams p;
+  p.w = a.w;
+  p.q_scale = a.q_scale;
+  p.k_scale = a.k_scale;
+  p.scores = a.scores;
+  p.ld = a.ld;
+  p.B = a.B;
+  p.T = a.T;
+  p.S = a.S;
+  p.q_begin = a.q_begin;
+  p.q_count = a.q_count;
+  p.nb = (a.q_count + QPS - 1) / QPS;
+  if (p.nb > kMaxNB) p.nb = kMaxNB;
+  const int per_group = p.nb * QPS;
+  p.groups_per_seq = (a.q_count + per_group - 1) / per_group;
+  p.spin = c.spin_limit;
+  p.err = c.err;
+  // count the items to size the grid
+  long long items = 0;
+  for (int g = 0; g < p.groups_per_seq; ++g) {
+    const int t0 = a.q_begin + g * per_group;
+    const int tend = t0 + per_group < a.q_begin + a.q_count ? t0 + per_group : a.q_begin + a.q_count;
+    const int ntiles = (a.S - a.T + tend - 1) / kBM + 1;
+    items += (ntiles + kKC - 1) / kKC;
+  }
+  items *= a.B;
+  const int grid = (int)(items < c.num_sms ? items : c.num_sms);
+  if (grid <= 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<DI, HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::kAlloc);
+  if (e != cudaSuccess) return e;
+  indexer_tc_kernel<DI, HI><<<grid, kThreads, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <int DI>
+cudaError_t launch_di(const LaunchCtx& c, const IndexerArgs& a) {
+  switch (a.H_I) {
+    case 4: return launch_tc<DI, 4>(c, a);
+    case 8: return launch_tc<DI, 8>(c, a);
+    case 16: return launch_tc<DI, 16>(c, a);
+    case 32: return launch_tc<DI, 32>(c, a);
+    case 64: return launch_tc<DI, 64>(c, a);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_indexer(const LaunchCtx& c, const IndexerArgs& a) {
   if (a.q_count <= 0 || a.B <= 0) return cudaSuccess;
-  const int last_pos = a.S - a.T + a.q_begin + a.q_count - 1;
-  dim3 grid((last_pos + kKeysPerBlock) / kKeysPerBlock, a.q_count, a.B);
-  size_t smem = (size_t)(a.H_I * a.D_I + a.H_I) * sizeof(float);
   switch (a.D_I) {
-    case 32: indexer_cuda_core_kernel<32><<<grid, kKeysPerBlock, smem, c.stream>>>(a); break;
-    case 64: indexer_cuda_core_kernel<64><<<grid, kKeysPerBlock, smem, c.stream>>>(a); break;
-    case 128: indexer_cuda_core_kernel<128><<<grid, kKeysPerBlock, smem, c.stream>>>(a); break;
+    case 32: return launch_di<32>(c, a);
+    case 64: return launch_di<64>(c, a);
+    case 128: return launch_di<128>(c, a);
     default: return cudaErrorInvalidValue;
   }
-  note_launches(1);
-  return cudaGetLastError();
 }
 
 }  // namespace dsa
