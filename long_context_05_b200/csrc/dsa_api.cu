@@ -20,7 +20,7 @@ void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::mem
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr long long kDefaultSpinLimit = 1LL << 26;  // about 0.1-1 s of polling
+constexpr long long kDefaultSpinLimit = 1LL << 22;  // polls per wait: well under a second
 long long g_spin_limit = kDefaultSpinLimit;
 
 struct DeviceInfo {

@@ -115,17 +115,6 @@ __device__ __forceinline__ bool subtile_active(const IdxParams& p, const Item& i
   return kt * kBM <= p.S - p.T + qlast;
 }
 
-__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
-        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-      :
-      : "memory");
-}
-
 template <int DI, int HI>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -177,6 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  const AbortSources ab{abort_flag, &p.err->code};
+  const AbortSources no_abort{nullptr, nullptr};  // drains of this CTA's own async work
   auto fail = [&](unsigned where) {
     report_error(p.err, DSA_ERR_TIMEOUT, ERR_SITE_INDEXER | (where << 8));
     *abort_flag = 1;
@@ -193,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kStages; ++i) issued[i] = false;
       bool ok = true;
       for_each_item<HI>(p, [&](const Item& it) {
-        if (!mbar_wait(b_empty, (items & 1) ^ 1, p.spin, abort_flag)) { fail(1); ok = false; return false; }
+        if (!mbar_wait(b_empty, (items & 1) ^ 1, p.spin, ab)) { fail(1); ok = false; return false; }
         int nsub = 0;
         for (int j = 0; j < p.nb; ++j)
           if (it.t0 + j * QPS < it.tend) nsub = j + 1;
@@ -204,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
-          if (!mbar_wait(&a_empty[st], ((a_cnt / kStages) & 1) ^ 1, p.spin, abort_flag)) {
+          if (!mbar_wait(&a_empty[st], ((a_cnt / kStages) & 1) ^ 1, p.spin, ab)) {
             fail(2); ok = false; return false;
           }
           mbar_arrive_expect_tx(&a_full[st], L::kABytes);
@@ -216,8 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       });
       // let every load this CTA started land before it exits
       for (int st = 0; st < kStages; ++st)
-        if (issued[st]) mbar_wait(&a_full[st], last_phase[st], p.spin, nullptr);
-      if (items > 0) mbar_wait(b_full, (items - 1) & 1, p.spin, nullptr);
+        if (issued[st]) mbar_wait(&a_full[st], last_phase[st], p.spin, no_abort);
+      if (items > 0) mbar_wait(b_full, (items - 1) & 1, p.spin, no_abort);
       (void)ok;
     }
   } else if (warp == 1) {
@@ -227,18 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t a_cnt = 0, items = 0, u = 0;
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
       for_each_item<HI>(p, [&](const Item& it) {
-        if (!mbar_wait(b_full, items & 1, p.spin, abort_flag)) { fail(3); return false; }
+        if (!mbar_wait(b_full, items & 1, p.spin, ab)) { fail(3); return false; }
         ++items;
         const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
-          if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.spin, abort_flag)) { fail(4); return false; }
+          if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.spin, ab)) { fail(4); return false; }
           tc_fence_after();
           const uint64_t adesc = make_sdesc(a_base + st * L::kABytes, 16, L::kSBO, L::kSwizzleLayout);
           for (int j = 0; j < p.nb; ++j) {
             if (!subtile_active<HI>(p, it, j, kt)) continue;
             const int acc = u % kNAcc;
-            if (!mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.spin, abort_flag)) { fail(5); return false; }
+            if (!mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.spin, ab)) { fail(5); return false; }
             tc_fence_after();
             const uint64_t bdesc = make_sdesc(b_base + j * L::kBSubBytes, 16, L::kSBO, L::kSwizzleLayout);
 #pragma unroll
@@ -253,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       });
       mma_commit(mma_done);
-      mbar_wait(mma_done, 0, p.spin, nullptr);
+      mbar_wait(mma_done, 0, p.spin, no_abort);
     }
   } else {
     // ---------------------------------------------------------- epilogue
@@ -276,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wbuf[x] = v;
       }
       mbar_arrive(&w_ready[items & 1]);
-      if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.spin, abort_flag)) { fail(7); return false; }
+      if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.spin, ab)) { fail(7); return false; }
       ++items;
       const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
       for (int kt = kt0; kt < kt1; ++kt) {
@@ -287,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t my = u++;
           if ((int)(my & 1) != grp) continue;
           const int acc = my % kNAcc;
-          if (!mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.spin, abort_flag)) { fail(6); return false; }
+          if (!mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.spin, ab)) { fail(6); return false; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kNSub;
           const float* wq = wbuf + j * kNSub;
