@@ -98,10 +98,11 @@ float tau_of(const dsa_shape* s) {
 }
 
 // Workspace layout (each region 256-byte aligned):
-//   [scores: B * q_rows * ld floats][attention split partials]
+//   [scores: B * q_rows * ld floats][attention split partials][top-k histograms]
 struct WsLayout {
   size_t scores_off, scores_bytes;
   size_t part_off, part_bytes;
+  size_t topk_off, topk_bytes;
   size_t total;
   int nsplit;
   int q_rows;
@@ -115,7 +116,10 @@ WsLayout ws_layout(const dsa_shape* s, int num_sms) {
   L.nsplit = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->k, num_sms) : 1;
   L.part_off = L.scores_off + L.scores_bytes;
   L.part_bytes = round_up(attn_partial_floats(s->B * s->T, s->H, s->d_v, L.nsplit) * sizeof(float), 256);
-  L.total = L.part_off + L.part_bytes;
+  L.topk_off = L.part_off + L.part_bytes;
+  const int topk_rows = s->B * L.q_rows;
+  L.topk_bytes = topk_uses_workspace(topk_rows, s->S, num_sms) ? round_up(topk_workspace_bytes(topk_rows), 256) : 0;
+  L.total = L.topk_off + L.topk_bytes;
   return L;
 }
 
@@ -133,12 +137,12 @@ dsa_status run_indexer(const LaunchCtx& c, const dsa_shape* s, const uint8_t* q_
 }
 
 dsa_status run_topk(const LaunchCtx& c, const dsa_shape* s, const float* scores, int64_t ld, int q_begin,
-                    int q_count, int32_t* idx) {
+                    int q_count, int32_t* idx, void* ws, size_t ws_bytes) {
   TopkArgs a;
   a.scores = scores; a.ld = ld; a.idx = idx;
   a.B = s->B; a.T = s->T; a.S = s->S; a.k = s->k;
   a.q_begin = q_begin; a.q_count = q_count;
-  return from_cuda(launch_topk(c, a));
+  return from_cuda(launch_topk(c, a, ws, ws_bytes));
 }
 
 dsa_status run_attn(const LaunchCtx& c, const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
@@ -209,15 +213,14 @@ dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_I, const floa
 
 dsa_status dsa_topk(const dsa_shape* s, const float* scores, int64_t ld_scores, int q_begin, int q_count,
                     int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws; (void)ws_bytes;
   dsa_status st = check_shape(s);
   if (st != DSA_OK) return st;
-  if (scores == nullptr || idx == nullptr) return DSA_ERR_INVALID_ARG;
+  if (scores == nullptr || idx == nullptr || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
   if (q_begin < 0 || q_count < 0 || q_begin + q_count > s->T) return DSA_ERR_INVALID_ARG;
-  if (ld_scores < s->S) return DSA_ERR_INVALID_ARG;
+  if (ld_scores < s->S || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
-  return run_topk(c, s, scores, ld_scores, q_begin, q_count, idx);
+  return run_topk(c, s, scores, ld_scores, q_begin, q_count, idx, ws, ws_bytes);
 }
 
 dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv, const int32_t* idx,
@@ -254,7 +257,9 @@ dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, 
     const int cnt = (s->T - q0) < L.q_rows ? (s->T - q0) : L.q_rows;
     if ((st = run_indexer(c, s, in->q_I, in->q_scale, in->w, in->k_I, in->k_scale, q0, cnt, scores, ld)) != DSA_OK)
       return st;
-    if ((st = run_topk(c, s, scores, ld, q0, cnt, idx_out)) != DSA_OK) return st;
+    if ((st = run_topk(c, s, scores, ld, q0, cnt, idx_out,
+                       L.topk_bytes ? static_cast<char*>(ws) + L.topk_off : nullptr, L.topk_bytes)) != DSA_OK)
+      return st;
   }
   return run_attn(c, s, in->q, in->kv, idx_out, out, lse, part, L.nsplit);
 }

@@ -75,7 +75,10 @@ struct AttnArgs {
 void note_launches(int n);
 
 cudaError_t launch_indexer(const LaunchCtx& c, const IndexerArgs& a);
-cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a);
+// ws: optional scratch for the split path (few long rows); see topk.cu
+cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t ws_bytes);
+size_t topk_workspace_bytes(int rows);
+bool topk_uses_workspace(int rows, int S, int num_sms);
 cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a);
 
 // split-k partial buffer size (floats) for a decode attention launch

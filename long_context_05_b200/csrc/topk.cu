@@ -5,116 +5,365 @@
 // key/value entries are kept, 2,048 per query; tenelement.pl, section
 // "Architektura ...", "Selekcja top-k" bullet).  The selection stays on the
 // device and reads the row straight from the score tile (sider.ai blog,
-// "Uyarilar": no CPU-GPU ping-pong in candidate selection).
+// "Uyarilar": candidate selection must not bounce between CPU and GPU and
+// must be cache-aware).
 //
-// Method: radix select on order-preserving 32-bit keys, one block per row.
-// Each pass histograms the next 8 bits of the keys that still match the
-// prefix found so far and picks the bucket holding the k-th largest key; after
-// four passes the k-th largest key `thr` is known exactly, together with how
-// many keys equal to it must be kept.  A last pass in index order writes every
-// key above `thr` and the lowest-indexed keys equal to it.
+// Keys: scores mapped to order-preserving 32-bit unsigned keys (-0.0 folded
+// onto +0.0).  Method, one block of 1024 threads per row:
+//   1. one pass over the row builds a 2048-bin histogram of the top 11 key
+//      bits; a block scan finds the bin B holding the k-th largest key;
+//   2. a second pass (the row is now in L2) writes every key above bin B to
+//      the output and copies the keys of bin B, with their indices, into
+//      shared memory;
+//   3. radix select over those candidates (8-bit digits) finds the exact k-th
+//      key `thr`; candidates above it are written, and of the candidates equal
+//      to it the lowest indices are kept (a second radix select on the bitwise
+//      complement of the index picks them).
+// If bin B holds more candidates than shared memory takes, steps 2-3 run as
+// radix passes over the row itself and a final pass in index order.
+// Decode rows (few, long) are split over several blocks for steps 1-2, with
+// the histogram and the candidates gathered in the caller's workspace.
 #include "internal.h"
 
 namespace dsa {
 namespace {
 
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;           // top 11 bits
+constexpr int kBinShift = 21;
+constexpr int kCap = 8192;            // candidates held in shared memory
+constexpr int kSegBlocks = 16;        // blocks per row in the split (decode) path
 
-// float -> unsigned with the same order; -0.0 is folded onto +0.0
 __device__ __forceinline__ unsigned int order_key(float f) {
   unsigned int u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_radix_kernel(TopkArgs a) {
-  __shared__ unsigned int hist[256];
-  __shared__ unsigned int s_digit, s_krem;
-  __shared__ int s_count, s_eq_base;
-  __shared__ int warp_eq[kTopkWarps];
-
-  const int r = blockIdx.x;
-  const int b = r / a.q_count;
-  const int i = r - b * a.q_count;
-  const int t = a.q_begin + i;
-  const int n = a.S - a.T + t + 1;  // visible keys
-  const int k = a.k;
-  const float* row = a.scores + (size_t)r * a.ld;
-  int32_t* out = a.idx + ((size_t)b * a.T + t) * k;
-  const int tid = threadIdx.x;
-
-  if (n <= k) {
-    for (int x = tid; x < k; x += kTopkThreads) out[x] = x < n ? x : -1;
-    return;
+// Block-wide inclusive scan of one value per thread; returns the inclusive
+// prefix and writes the block total to *total.
+__device__ __forceinline__ unsigned int block_scan(unsigned int v, unsigned int* warp_tot, unsigned int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-
-  unsigned int prefix = 0u, mask = 0u;
-  unsigned int krem = (unsigned int)k;  // rank of the wanted key among the matching ones
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int x = tid; x < 256; x += kTopkThreads) hist[x] = 0u;
-    __syncthreads();
-    for (int x = tid; x < n; x += kTopkThreads) {
-      const unsigned int key = order_key(row[x]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned int w = warp_tot[lane];
+    unsigned int s = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
     }
-    __syncthreads();
-    if (tid == 0) {
-      unsigned int cum = 0u;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (cum + hist[d] >= krem) break;
-        cum += hist[d];
-      }
-      s_digit = (unsigned int)d;
-      s_krem = krem - cum;
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    mask |= 255u << shift;
-    krem = s_krem;
-    __syncthreads();
-  }
-  const unsigned int thr = prefix;  // the k-th largest key; keep krem copies of it
-
-  if (tid == 0) {
-    s_count = 0;
-    s_eq_base = 0;
+    warp_tot[lane] = s - w;  // exclusive prefix of the warps
+    if (lane == 31) *total = s;
   }
   __syncthreads();
+  const unsigned int r = x + warp_tot[warp];
+  __syncthreads();
+  return r;
+}
+
+// Find the bin holding the rank-th largest key (rank >= 1) among bins
+// counted in hist[0..nb) (nb = kBins or 256; larger bin = larger keys).
+// Returns the bin in *bin and the count of keys in higher bins in *above.
+__device__ void find_bin(const unsigned int* hist, int nb, unsigned int rank, unsigned int* warp_tot,
+                         unsigned int* s_bin, unsigned int* s_above, unsigned int* s_total) {
+  const int per = nb / kThreads > 0 ? nb / kThreads : 1;  // 2 for kBins, 1 for 256
+  unsigned int local = 0;
+  unsigned int c[2] = {0u, 0u};
+  const int t = threadIdx.x;
+  // thread t owns bins nb-1-per*t ... (descending)
+  if (t * per < nb) {
+    for (int i = 0; i < per; ++i) {
+      c[i] = hist[nb - 1 - (per * t + i)];
+      local += c[i];
+    }
+  }
+  const unsigned int incl = block_scan(local, warp_tot, s_total);
+  const unsigned int excl = incl - local;
+  if (t * per < nb && excl < rank && incl >= rank) {
+    unsigned int run = excl;
+    for (int i = 0; i < per; ++i) {
+      if (run + c[i] >= rank) {
+        *s_bin = (unsigned int)(nb - 1 - (per * t + i));
+        *s_above = run;
+        break;
+      }
+      run += c[i];
+    }
+  }
+  __syncthreads();
+}
+
+// Radix select over `count` keys delivered by key_of(i) that all share the bits
+// in `mask` with `prefix`: finds the rank-th largest key (rank >= 1), refining
+// 8 bits at a time from bit `hi` down to bit 0.  Returns the key; *krem gets
+// how many keys equal to it belong to the top `rank`.
+template <class KeyOf>
+__device__ unsigned int radix_select(KeyOf key_of, int count, unsigned int prefix, unsigned int mask, int hi,
+                                     unsigned int rank, unsigned int* hist, unsigned int* warp_tot,
+                                     unsigned int* s_bin, unsigned int* s_above, unsigned int* s_total,
+                                     unsigned int* krem_out) {
+  unsigned int krem = rank;
+  while (hi > 0) {
+    const int bits = hi >= 8 ? 8 : hi;
+    const int shift = hi - bits;
+    const unsigned int dmask = (1u << bits) - 1u;
+    for (int x = threadIdx.x; x < 256; x += kThreads) hist[x] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < count; i += kThreads) {
+      const unsigned int key = key_of(i);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    find_bin(hist, 256, krem, warp_tot, s_bin, s_above, s_total);
+    prefix |= *s_bin << shift;
+    mask |= dmask << shift;
+    krem -= *s_above;
+    hi = shift;
+    __syncthreads();
+  }
+  *krem_out = krem;
+  return prefix;
+}
+
+struct Smem {
+  unsigned int hist[kBins];
+  unsigned int ck[kCap];  // candidate keys
+  int ci[kCap];           // candidate indices
+  int eqi[kCap];          // indices of the candidates equal to the k-th key
+  unsigned int warp_tot[kWarps];
+  unsigned int bin, above, total, krem2;
+  int cnt, ncand, eq_base;
+  int warp_eq[kWarps];
+};
+
+// Steps 2-3 on a row whose threshold bin B (and the count above it) is known.
+// keys_in_bin: number of keys in bin B over the whole row.
+__device__ void select_from_bin(const float* row, int n, int k, int32_t* out, unsigned int B, unsigned int above,
+                                unsigned int keys_in_bin, Smem& sm) {
+  const int tid = threadIdx.x;
+  const unsigned int need = (unsigned int)k - above;  // keys to take from bin B (>= 1)
+  if (tid == 0) {
+    sm.cnt = 0;
+    sm.ncand = 0;
+  }
+  __syncthreads();
+  const bool fits = keys_in_bin <= (unsigned int)kCap;
+  // pass 2: keys above bin B go straight out; bin B keys become candidates
+  for (int x = tid; x < n; x += kThreads) {
+    const unsigned int key = order_key(row[x]);
+    const unsigned int bin = key >> kBinShift;
+    if (bin > B) {
+      out[atomicAdd(&sm.cnt, 1)] = x;
+    } else if (bin == B && fits) {
+      const int p = atomicAdd(&sm.ncand, 1);
+      sm.ck[p] = key;
+      sm.ci[p] = x;
+    }
+  }
+  __syncthreads();
+  unsigned int thr, krem;
+  if (fits) {
+    const int nc = sm.ncand;
+    const unsigned int* ck = sm.ck;
+    thr = radix_select([ck](int i) { return ck[i]; }, nc, B << kBinShift, 0xFFFFFFFFu << kBinShift, kBinShift,
+                       need, sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
+    // candidates above thr
+    unsigned int eq_local = 0;
+    for (int i = tid; i < nc; i += kThreads) {
+      if (sm.ck[i] > thr) out[atomicAdd(&sm.cnt, 1)] = sm.ci[i];
+      eq_local += sm.ck[i] == thr;
+    }
+    block_scan(eq_local, sm.warp_tot, &sm.total);
+    const unsigned int E = sm.total;
+    if (E == krem) {
+      for (int i = tid; i < nc; i += kThreads)
+        if (sm.ck[i] == thr) out[atomicAdd(&sm.cnt, 1)] = sm.ci[i];
+      return;
+    }
+    // more equal keys than slots: keep the lowest indices.  Gather the equal
+    // candidates' indices and select on ~index (lower index = larger key).
+    if (tid == 0) sm.eq_base = 0;
+    __syncthreads();
+    for (int i = tid; i < nc; i += kThreads)
+      if (sm.ck[i] == thr) sm.eqi[atomicAdd(&sm.eq_base, 1)] = sm.ci[i];
+    __syncthreads();
+    const int ne = sm.eq_base;
+    const int* ci = sm.eqi;
+    unsigned int krem2;
+    const unsigned int ithr = radix_select([ci](int i) { return ~(unsigned int)ci[i]; }, ne, 0u, 0u, 32, krem,
+                                           sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem2);
+    for (int i = tid; i < ne; i += kThreads)
+      if (~(unsigned int)sm.eqi[i] >= ithr) out[atomicAdd(&sm.cnt, 1)] = sm.eqi[i];
+    return;
+  }
+  // bin B too large for shared memory: radix passes over the row itself
+  thr = radix_select([row](int i) { return order_key(row[i]); }, n, B << kBinShift, 0xFFFFFFFFu << kBinShift,
+                     kBinShift, need, sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
+  // keys in bin B above thr, then the krem lowest-indexed keys equal to thr
+  if (tid == 0) sm.eq_base = 0;
+  __syncthreads();
   const int lane = tid & 31, warp = tid >> 5;
-  for (int base = 0; base < n; base += kTopkThreads) {
+  for (int base = 0; base < n; base += kThreads) {
     const int x = base + tid;
     const bool valid = x < n;
     const unsigned int key = valid ? order_key(row[x]) : 0u;
-    const bool gt = valid && key > thr;
+    if (valid && (key >> kBinShift) == B && key > thr) out[atomicAdd(&sm.cnt, 1)] = x;
     const bool eq = valid && key == thr;
-    if (gt) out[atomicAdd(&s_count, 1)] = x;
     const unsigned int bal = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) warp_eq[warp] = __popc(bal);
+    if (lane == 0) sm.warp_eq[warp] = __popc(bal);
     __syncthreads();
-    int before = s_eq_base;
-    for (int w = 0; w < warp; ++w) before += warp_eq[w];
+    int before = sm.eq_base;
+    for (int w = 0; w < warp; ++w) before += sm.warp_eq[w];
     before += __popc(bal & ((1u << lane) - 1u));
-    if (eq && before < (int)krem) out[atomicAdd(&s_count, 1)] = x;
+    if (eq && before < (int)krem) out[atomicAdd(&sm.cnt, 1)] = x;
     __syncthreads();
     if (tid == 0) {
       int tot = 0;
-      for (int w = 0; w < kTopkWarps; ++w) tot += warp_eq[w];
-      s_eq_base += tot;
+      for (int w = 0; w < kWarps; ++w) tot += sm.warp_eq[w];
+      sm.eq_base += tot;
     }
     __syncthreads();
   }
 }
 
+__device__ __forceinline__ void row_setup(const TopkArgs& a, int r, int* b, int* t, int* n, const float** row,
+                                          int32_t** out) {
+  *b = r / a.q_count;
+  const int i = r - *b * a.q_count;
+  *t = a.q_begin + i;
+  *n = a.S - a.T + *t + 1;
+  *row = a.scores + (size_t)r * a.ld;
+  *out = a.idx + ((size_t)*b * a.T + *t) * a.k;
+}
+
+__device__ void histogram_pass(const float* row, int lo, int hi, unsigned int* hist) {
+  // vectorised over the 16-byte aligned middle of [lo, hi)
+  const int a0 = (lo + 3) & ~3, a1 = hi & ~3;
+  if (a0 >= a1) {
+    for (int x = lo + (int)threadIdx.x; x < hi; x += kThreads) atomicAdd(&hist[order_key(row[x]) >> kBinShift], 1u);
+    return;
+  }
+  for (int x = lo + (int)threadIdx.x; x < a0; x += kThreads) atomicAdd(&hist[order_key(row[x]) >> kBinShift], 1u);
+  const float4* r4 = reinterpret_cast<const float4*>(row + a0);
+  for (int x = threadIdx.x; x < (a1 - a0) / 4; x += kThreads) {
+    const float4 v = r4[x];
+    atomicAdd(&hist[order_key(v.x) >> kBinShift], 1u);
+    atomicAdd(&hist[order_key(v.y) >> kBinShift], 1u);
+    atomicAdd(&hist[order_key(v.z) >> kBinShift], 1u);
+    atomicAdd(&hist[order_key(v.w) >> kBinShift], 1u);
+  }
+  for (int x = a1 + (int)threadIdx.x; x < hi; x += kThreads) atomicAdd(&hist[order_key(row[x]) >> kBinShift], 1u);
+}
+
+// One block per row.
+__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(TopkArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, blockIdx.x, &b, &t, &n, &row, &out);
+  const int k = a.k;
+  if (n <= k) {
+    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
+    return;
+  }
+  for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = 0u;
+  __syncthreads();
+  histogram_pass(row, 0, n, sm.hist);
+  __syncthreads();
+  find_bin(sm.hist, kBins, (unsigned int)k, sm.warp_tot, &sm.bin, &sm.above, &sm.total);
+  const unsigned int B = sm.bin, above = sm.above, inbin = sm.hist[B];
+  __syncthreads();
+  select_from_bin(row, n, k, out, B, above, inbin, sm);
+}
+
+// ---------------------------------------------------------------- split path
+// Workspace per row: hist[kBins] u32.  Kernel 1 adds each segment's histogram;
+// kernel 2 (one block per row) finds the bin and runs steps 2-3.
+
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist) {
+  __shared__ unsigned int hist[kBins];
+  const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, r, &b, &t, &n, &row, &out);
+  if (n <= a.k) return;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) hist[x] = 0u;
+  __syncthreads();
+  const int per = ((n + kSegBlocks - 1) / kSegBlocks + 3) & ~3;
+  const int lo = seg * per, hi = min(n, lo + per);
+  if (lo < hi) histogram_pass(row, lo, hi, hist);
+  __syncthreads();
+  unsigned int* gh = ghist + (size_t)r * kBins;
+  for (int x = threadIdx.x; x < kBins; x += kThreads)
+    if (hist[x]) atomicAdd(&gh[x], hist[x]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_select_kernel(TopkArgs a, unsigned int* ghist) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, blockIdx.x, &b, &t, &n, &row, &out);
+  const int k = a.k;
+  if (n <= k) {
+    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
+    return;
+  }
+  unsigned int* gh = ghist + (size_t)blockIdx.x * kBins;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = gh[x];
+  __syncthreads();
+  find_bin(sm.hist, kBins, (unsigned int)k, sm.warp_tot, &sm.bin, &sm.above, &sm.total);
+  const unsigned int B = sm.bin, above = sm.above, inbin = sm.hist[B];
+  __syncthreads();
+  select_from_bin(row, n, k, out, B, above, inbin, sm);
+}
+
+__global__ void topk_zero_kernel(unsigned int* p, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0u;
+}
+
 }  // namespace
 
-cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a) {
+size_t topk_workspace_bytes(int rows) { return (size_t)rows * kBins * sizeof(unsigned int); }
+
+bool topk_uses_workspace(int rows, int S, int num_sms) { return rows * 2 < num_sms && S >= 16 * kThreads; }
+
+cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t ws_bytes) {
   const int rows = a.B * a.q_count;
   if (rows <= 0) return cudaSuccess;
-  topk_radix_kernel<<<rows, kTopkThreads, 0, c.stream>>>(a);
+  const size_t smem = sizeof(Smem);
+  cudaError_t e;
+  // few long rows: split the histogram pass over several blocks per row
+  const bool split =
+      ws != nullptr && ws_bytes >= topk_workspace_bytes(rows) && topk_uses_workspace(rows, a.S, c.num_sms);
+  if (!split) {
+    e = cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_row_kernel<<<rows, kThreads, smem, c.stream>>>(a);
+    note_launches(1);
+    return cudaGetLastError();
+  }
+  unsigned int* gh = static_cast<unsigned int*>(ws);
+  topk_zero_kernel<<<64, 256, 0, c.stream>>>(gh, (size_t)rows * kBins);
   note_launches(1);
+  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, gh);
+  e = cudaFuncSetAttribute(topk_seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_seg_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, gh);
+  note_launches(2);
   return cudaGetLastError();
 }
 
