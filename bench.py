@@ -38,6 +38,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from long_context_05_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+from long_context_05_b200.parallel import barrier as _barrier, max_over_ranks as _max_over_ranks  # noqa: E402
+from long_context_05_b200.parallel import rank_seed  # noqa: E402
 
 METRIC = "DSA tokens/s (prefill, decode) at 128K ctx; % of HBM / tensor-core roofline"
 PREFILL = "prefill_128k"
@@ -74,17 +76,11 @@ def dist_setup(n_gpus):
 
 def barrier(ws):
     if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+        _barrier(torch.device("cuda", torch.cuda.current_device()))
 
 
 def max_over_ranks(x, ws):
-    if ws <= 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _max_over_ranks(x, device="cuda") if ws > 1 else x
 
 
 class ClockSampler:
@@ -171,7 +167,7 @@ class DsaRunner:
     def __init__(self, wl, seed_offset=0):
         from long_context_05_b200 import dsa
         self.dsa = dsa
-        self.wl = wl = wl.with_(seed=wl.seed + seed_offset)
+        self.wl = wl = wl.with_(seed=rank_seed(wl.seed, seed_offset))
         self.inp = make_inputs(wl, "cuda")
         self.inp.pop("needle_pos", None)
         self.shape = dsa.make_shape(wl)

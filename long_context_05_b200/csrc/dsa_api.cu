@@ -20,7 +20,7 @@ void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::mem
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr long long kDefaultSpinLimit = 1LL << 22;  // polls per wait: well under a second
+constexpr long long kDefaultSpinLimit = 1LL << 25;  // polls per wait before giving up
 long long g_spin_limit = kDefaultSpinLimit;
 
 struct DeviceInfo {

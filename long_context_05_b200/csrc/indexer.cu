@@ -278,7 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t my = u++;
           if ((int)(my & 1) != grp) continue;
           const int acc = my % kNAcc;
-          if (!mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.spin, ab)) { fail(6); return false; }
+          const bool got = mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.spin, ab);
+          if (!__all_sync(0xffffffffu, got)) { fail(6); return false; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kNSub;
           const float* wq = wbuf + j * kNSub;

@@ -99,7 +99,11 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 // ------------------------------------------------------------------ TMEM
 
 // Warp-wide: allocate ncols TMEM columns; the base address lands in *dst (smem).
+// The tcgen05 .sync.aligned instructions (alloc, dealloc, ld, st, wait) need
+// the whole warp converged: callers reconverge with __syncwarp() after any
+// lane-divergent code (per-lane waits, lane-0 work) before issuing them.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  __syncwarp();
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
                : "memory");
 }
@@ -109,6 +113,7 @@ __device__ __forceinline__ void tmem_relinquish() {
 }
 
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  __syncwarp();
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
@@ -257,7 +262,10 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   return out;
 }
 
+// Every thread of both CTAs; the warp is reconverged first because the
+// .aligned forms require all lanes of a warp to execute them together.
 __device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 

@@ -276,6 +276,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           c = qsrc[2 * g + 1];
         }
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        __syncwarp();
         tmem_st8(tmem + lane_addr + kQCol + g * 8, w);
       }
       tmem_wait_st();
@@ -394,6 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int c = 0; c < C::DVH / 32; ++c) {
           uint32_t o[32];
+          __syncwarp();
           tmem_ld32(tmem + lane_addr + kOCol + c * 32, o);
           tmem_wait_ld_dep(o);
 #pragma unroll
@@ -420,6 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int vlo = C::v_lo(rank);
       for (int c = 0; c < C::DVH / 32; ++c) {
         uint32_t o[32];
+        __syncwarp();
         tmem_ld32(tmem + lane_addr + kOCol + c * 32, o);
         tmem_wait_ld_dep(o);
         if (!write_o) continue;
