@@ -73,7 +73,7 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_META + kStages * kN;
   static constexpr int NBARS = 2 * kStages + 1 + 2 + 2 + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int BYTES = OFF_MISC + 32;
   static constexpr int ALLOC = BYTES + 1024;
   static_assert(DVH <= 256 && DVH % 16 == 0, "value columns per CTA");
   static_assert(KS0 * 8 + kQCol <= kTmemCols, "Q half must fit in TMEM");
@@ -122,6 +122,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = peer_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  // chunk each role is on (diagnostics for a timeout): producer, MMA, softmax
+  volatile int* prog = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -150,6 +152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
+    prog[0] = prog[1] = prog[2] = 0;
     fence_mbar_init();
     // arm the first two exchange phases before the peer can write
     mbar_arrive_expect_tx(&x_full[0], C::X_BYTES);
@@ -166,8 +169,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   const AbortSources ab{abort_flag, &p.err->code};
   const AbortSources no_abort{nullptr, nullptr};  // drains of this CTA's own async work
+  // detail: site | where << 8 | rank << 12 | producer, MMA, softmax chunk (6 bits each)
   auto fail = [&](unsigned where) {
-    report_error(p.err, DSA_ERR_TIMEOUT, ERR_SITE_ATTN | (where << 8));
+    const unsigned d = ERR_SITE_ATTN | ((where & 15u) << 8) | (rank << 12) | ((unsigned)(prog[0] & 63) << 13) |
+                       ((unsigned)(prog[1] & 63) << 19) | ((unsigned)(prog[2] & 63) << 25);
+    report_error(p.err, DSA_ERR_TIMEOUT, d);
     *abort_flag = 1;
   };
   const int atom_lo = C::atom_lo(rank);
@@ -182,6 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nchunks && ok; ++j) {
       const int st = j % kStages;
+      if (pt == 0) prog[0] = j;
       if (!mbar_wait(&kv_empty[st], ((j / kStages) & 1) ^ 1, p.spin, ab)) { fail(1); ok = false; break; }
       uint8_t* stage = sKV + st * C::STAGE_BYTES;
 #pragma unroll
@@ -242,6 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       for (int j = 0; j < nchunks && ok; ++j) {
         const int st = j % kStages;
+        prog[1] = j;
         if (!mbar_wait(&kv_full[st], (j / kStages) & 1, p.spin, ab)) { fail(4); ok = false; break; }
         fence_proxy_async_smem();
         if (j >= 1 && !mbar_wait(&s_free[0], (j - 1) & 1, p.spin, ab)) { fail(5); ok = false; break; }
@@ -298,6 +306,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nchunks && ok; ++j) {
       const int bsel = j & 1;
+      if (threadIdx.x == kSoftWarp0 * 32) prog[2] = j;
       // 1. partial logits of this CTA
       if (!wwait(&s_full[0], j & 1, false)) { fail(6); ok = false; break; }
       tc_fence_after();
