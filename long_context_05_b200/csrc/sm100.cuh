@@ -281,6 +281,13 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remot
       : "memory");
 }
 
+// Plain 16-byte store into another CTA's shared memory (shared::cluster
+// address); made visible to the peer by a later release arrive.
+__device__ __forceinline__ void st_cluster_v4(uint32_t remote_addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote_addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }

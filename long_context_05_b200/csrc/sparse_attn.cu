@@ -14,8 +14,9 @@
 //   * the key dimension of Q.K^T is halved: CTA r keeps its half of Q in TMEM
 //     (the A operand) and computes a partial logit tile S_r = Q_r K_r^T;
 //   * the two partial tiles are exchanged through distributed shared memory
-//     (st.async with mbarrier transaction counts) and both CTAs form the same
-//     S = S_0 + S_1, so both take identical softmax decisions;
+//     (plain shared::cluster stores published by a release arrive on the
+//     peer's mbarrier) and both CTAs form the same S = S_0 + S_1, so both take
+//     identical softmax decisions;
 //   * each CTA multiplies P by its half of V (256 of the 512 value columns)
 //     and owns that half of the output.
 // Keys arrive in chunks of 64 selected rows gathered with 16-byte cp.async
@@ -117,7 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* s_free = s_full + 2;        // [2]: index 0 used
   uint64_t* p_full = s_free + 2;        // [2]
   uint64_t* pv_done = p_full + 2;       // [2]
-  uint64_t* x_full = pv_done + 2;       // [2]: peer's partial logits landed (tx)
+  uint64_t* x_full = pv_done + 2;       // [2]: peer's partial logits landed (128 remote arrivals)
   uint64_t* peer_free = x_full + 2;     // [2]: peer consumed what we wrote
   uint64_t* mma_done = peer_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -147,16 +148,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
-      mbar_init(&x_full[i], 1);
+      mbar_init(&x_full[i], 128);
       mbar_init(&peer_free[i], 128);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     prog[0] = prog[1] = prog[2] = 0;
     fence_mbar_init();
-    // arm the first two exchange phases before the peer can write
-    mbar_arrive_expect_tx(&x_full[0], C::X_BYTES);
-    mbar_arrive_expect_tx(&x_full[1], C::X_BYTES);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -323,14 +321,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fail(7); ok = false; break;
       }
       const uint32_t xrow = xpeer + (uint32_t)(bsel * C::X_BYTES + h * kN * 4);
-      const uint32_t xbar = xfull_peer + bsel * 8;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const int v = (c < 8) ? 0 : 1;
         const int e = (c & 7) * 4;
-        st_async_v4(xrow + (uint32_t)((c ^ hs) * 16), xbar, __uint_as_float(sr[v][e]), __uint_as_float(sr[v][e + 1]),
-                    __uint_as_float(sr[v][e + 2]), __uint_as_float(sr[v][e + 3]));
+        st_cluster_v4(xrow + (uint32_t)((c ^ hs) * 16), __uint_as_float(sr[v][e]), __uint_as_float(sr[v][e + 1]),
+                      __uint_as_float(sr[v][e + 2]), __uint_as_float(sr[v][e + 3]));
       }
+      mbar_arrive_remote(xfull_peer + bsel * 8);  // release: the stores above are visible first
       // 3. add the peer's partial logits
       if (!wwait(&x_full[bsel], (j >> 1) & 1, true)) { fail(8); ok = false; break; }
       float s[kN];
@@ -345,10 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         s[4 * c + 2] = __uint_as_float(sr[v][e + 2]) + x.z;
         s[4 * c + 3] = __uint_as_float(sr[v][e + 3]) + x.w;
       }
-      if (j + 2 < nchunks) {
-        if (threadIdx.x == kSoftWarp0 * 32) mbar_arrive_expect_tx(&x_full[bsel], C::X_BYTES);
-        mbar_arrive_remote(pfree_peer + bsel * 8);
-      }
+      if (j + 2 < nchunks) mbar_arrive_remote(pfree_peer + bsel * 8);
       // 4. mask the empty slots, update the running maximum
       const int st = j % kStages;
       if (!wwait(&kv_full[st], (j / kStages) & 1, false)) { fail(9); ok = false; break; }
