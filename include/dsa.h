@@ -174,10 +174,11 @@ DSA_API dsa_status dsa_get_device_error(void* stream, int* detail);
  * or one timed region made. */
 DSA_API unsigned long long dsa_launch_count(void);
 
-/* Test hook for the bounded waits: sets the spin limit (iterations) every
- * later launch passes to its waits; 0 restores the default.  A tiny limit
- * makes waits give up early and report DSA_ERR_TIMEOUT instead of hanging. */
-DSA_API void dsa_set_spin_limit(long long iterations);
+/* Bounded waits: every wait inside a kernel gives up after this many
+ * microseconds of wall-clock time (default 2,000,000 = 2 s) and the kernel
+ * reports DSA_ERR_TIMEOUT instead of hanging.  Applies to later launches;
+ * values <= 0 restore the default.  A small value is a test hook. */
+DSA_API void dsa_set_wait_timeout_us(long long microseconds);
 
 #ifdef __cplusplus
 }

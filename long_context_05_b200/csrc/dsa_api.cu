@@ -20,8 +20,8 @@ void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::mem
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr long long kDefaultSpinLimit = 1LL << 25;  // polls per wait before giving up
-long long g_spin_limit = kDefaultSpinLimit;
+constexpr long long kDefaultWaitNs = 2000000000LL;  // 2 s per bounded wait
+long long g_wait_ns = kDefaultWaitNs;
 
 struct DeviceInfo {
   DevErr* err = nullptr;
@@ -57,7 +57,7 @@ dsa_status make_ctx(void* stream, LaunchCtx* c) {
   if (st != DSA_OK) return st;
   c->stream = static_cast<cudaStream_t>(stream);
   c->err = d.err;
-  c->spin_limit = g_spin_limit;
+  c->wait_ns = g_wait_ns;
   c->num_sms = d.num_sms;
   c->device = dev;
   return DSA_OK;
@@ -184,8 +184,8 @@ const char* dsa_status_string(dsa_status st) {
 
 unsigned long long dsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-void dsa_set_spin_limit(long long iterations) {
-  g_spin_limit = iterations > 0 ? iterations : kDefaultSpinLimit;
+void dsa_set_wait_timeout_us(long long microseconds) {
+  g_wait_ns = microseconds > 0 ? microseconds * 1000LL : kDefaultWaitNs;
 }
 
 size_t dsa_workspace_size(const dsa_shape* s) {

@@ -51,7 +51,7 @@ struct IdxParams {
   int B, T, S, q_begin, q_count;
   int nb;              // B sub-tiles per item
   int groups_per_seq;  // query groups per sequence
-  long long spin;
+  long long wait_ns;
   DevErr* err;
 };
 
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kStages; ++i) issued[i] = false;
       bool ok = true;
       for_each_item<HI>(p, [&](const Item& it) {
-        if (!mbar_wait(b_empty, (items & 1) ^ 1, p.spin, ab)) { fail(1); ok = false; return false; }
+        if (!mbar_wait(b_empty, (items & 1) ^ 1, p.wait_ns, ab)) { fail(1); ok = false; return false; }
         int nsub = 0;
         for (int j = 0; j < p.nb; ++j)
           if (it.t0 + j * QPS < it.tend) nsub = j + 1;
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
-          if (!mbar_wait(&a_empty[st], ((a_cnt / kStages) & 1) ^ 1, p.spin, ab)) {
+          if (!mbar_wait(&a_empty[st], ((a_cnt / kStages) & 1) ^ 1, p.wait_ns, ab)) {
             fail(2); ok = false; return false;
           }
           mbar_arrive_expect_tx(&a_full[st], L::kABytes);
@@ -207,8 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       });
       // let every load this CTA started land before it exits
       for (int st = 0; st < kStages; ++st)
-        if (issued[st]) mbar_wait(&a_full[st], last_phase[st], p.spin, no_abort);
-      if (items > 0) mbar_wait(b_full, (items - 1) & 1, p.spin, no_abort);
+        if (issued[st]) mbar_wait(&a_full[st], last_phase[st], p.wait_ns, no_abort);
+      if (items > 0) mbar_wait(b_full, (items - 1) & 1, p.wait_ns, no_abort);
       (void)ok;
     }
   } else if (warp == 1) {
@@ -218,18 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t a_cnt = 0, items = 0, u = 0;
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
       for_each_item<HI>(p, [&](const Item& it) {
-        if (!mbar_wait(b_full, items & 1, p.spin, ab)) { fail(3); return false; }
+        if (!mbar_wait(b_full, items & 1, p.wait_ns, ab)) { fail(3); return false; }
         ++items;
         const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
-          if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.spin, ab)) { fail(4); return false; }
+          if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.wait_ns, ab)) { fail(4); return false; }
           tc_fence_after();
           const uint64_t adesc = make_sdesc(a_base + st * L::kABytes, 16, L::kSBO, L::kSwizzleLayout);
           for (int j = 0; j < p.nb; ++j) {
             if (!subtile_active<HI>(p, it, j, kt)) continue;
             const int acc = u % kNAcc;
-            if (!mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.spin, ab)) { fail(5); return false; }
+            if (!mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.wait_ns, ab)) { fail(5); return false; }
             tc_fence_after();
             const uint64_t bdesc = make_sdesc(b_base + j * L::kBSubBytes, 16, L::kSBO, L::kSwizzleLayout);
 #pragma unroll
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       });
       mma_commit(mma_done);
-      mbar_wait(mma_done, 0, p.spin, no_abort);
+      mbar_wait(mma_done, 0, p.wait_ns, no_abort);
     }
   } else {
     // ---------------------------------------------------------- epilogue
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wbuf[x] = v;
       }
       mbar_arrive(&w_ready[items & 1]);
-      if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.spin, ab)) { fail(7); return false; }
+      if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.wait_ns, ab)) { fail(7); return false; }
       ++items;
       const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
       for (int kt = kt0; kt < kt1; ++kt) {
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t my = u++;
           if ((int)(my & 1) != grp) continue;
           const int acc = my % kNAcc;
-          const bool got = mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.spin, ab);
+          const bool got = mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.wait_ns, ab);
           if (!__all_sync(0xffffffffu, got)) { fail(6); return false; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kNSub;
@@ -359,7 +359,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   if (p.nb > kMaxNB) p.nb = kMaxNB;
   const int per_group = p.nb * QPS;
   p.groups_per_seq = (a.q_count + per_group - 1) / per_group;
-  p.spin = c.spin_limit;
+  p.wait_ns = c.wait_ns;
   p.err = c.err;
   // count the items to size the grid
   long long items = 0;

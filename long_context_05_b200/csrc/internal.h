@@ -34,7 +34,7 @@ __device__ __forceinline__ void report_error(DevErr* e, unsigned int code, unsig
 struct LaunchCtx {
   cudaStream_t stream;
   DevErr* err;            // device address of this device's error word
-  long long spin_limit;   // iterations before a bounded wait gives up
+  long long wait_ns;      // wall-clock limit of a bounded wait
   int num_sms;
   int device;
 };

@@ -1,8 +1,9 @@
 // Thin inline-PTX wrappers for the Blackwell (sm_100a) features the kernels
 // use: mbarriers with bounded waits, TMA tile loads, tcgen05 MMA / TMEM.
 //
-// Every wait in this library is bounded: it polls at most `limit` times and
-// then returns false, and the caller records DSA_ERR_TIMEOUT and unwinds.
+// Every wait in this library is bounded: it gives up after a wall-clock limit
+// (nanoseconds, %globaltimer) and returns false, and the caller records
+// DSA_ERR_TIMEOUT and unwinds.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -50,22 +51,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Where a wait looks for a reason to give up early: the CTA's own abort flag
-// (shared memory) and the device-wide error word (any CTA that timed out).
+// (shared memory, checked every 1024 polls) and the device-wide error word
+// (global memory, read only after the wait has lasted 1 ms and then only
+// every 65536 polls, so spinning threads never turn it into a hot spot).
 struct AbortSources {
   volatile int* cta;
   const volatile unsigned int* device;
-  __device__ __forceinline__ bool raised() const {
-    return (cta != nullptr && *cta != 0) || (device != nullptr && *device != 0u);
-  }
 };
 
-// Wait for the phase with the given parity to complete; false after `limit`
-// unsuccessful polls, or as soon as an abort source is raised.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit, AbortSources ab) {
-  for (long long i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63 && (i >= limit || ab.raised())) return false;
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete.  Returns false once
+// the wait has lasted `limit_ns` nanoseconds, or when an abort source is
+// raised.
+template <class TryWait>
+__device__ __forceinline__ bool bounded_wait(TryWait try_wait, long long limit_ns, AbortSources ab) {
+  if (try_wait()) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (try_wait()) return true;
+    if ((i & 1023u) == 0u) {
+      if (ab.cta != nullptr && *ab.cta != 0) return false;
+      const long long dt = (long long)(global_ns() - t0);
+      if (dt > limit_ns) return false;
+      if (ab.device != nullptr && dt > 1000000 && (i & 65535u) == 0u && *ab.device != 0u) return false;
+    }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_ns, AbortSources ab) {
+  return bounded_wait([&] { return mbar_try_wait(bar, parity); }, limit_ns, ab);
 }
 
 // ------------------------------------------------------------------ fences
@@ -305,12 +324,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 // Bounded wait with cluster-scope acquire (data written by the peer CTA).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long limit,
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long limit_ns,
                                                   AbortSources ab) {
-  for (long long i = 0;; ++i) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 63) == 63 && (i >= limit || ab.raised())) return false;
-  }
+  return bounded_wait([&] { return mbar_try_wait_cluster(bar, parity); }, limit_ns, ab);
 }
 
 __device__ __forceinline__ uint32_t elect_one() {

@@ -91,7 +91,7 @@ struct AttnParams {
   int T, S, H, k;
   int nsplit, kc;   // splits per row and selected slots per split
   float scale_log2; // tau * log2(e)
-  long long spin;
+  long long wait_ns;
   DevErr* err;
 };
 
@@ -187,7 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nchunks && ok; ++j) {
       const int st = j % kStages;
       if (pt == 0) prog[0] = j;
-      if (!mbar_wait(&kv_empty[st], ((j / kStages) & 1) ^ 1, p.spin, ab)) { fail(1); ok = false; break; }
+      if (!mbar_wait(&kv_empty[st], ((j / kStages) & 1) ^ 1, p.wait_ns, ab)) { fail(1); ok = false; break; }
       uint8_t* stage = sKV + st * C::STAGE_BYTES;
 #pragma unroll
       for (int m = 0; m < kN / 8; ++m) {
@@ -228,7 +228,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int nks = C::ks_of(rank);
       const uint32_t kv_base = smem_u32(sKV), p_base = smem_u32(sP);
       auto do_pv = [&](int i) -> bool {
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.spin, ab)) { fail(2); return false; }
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, p.wait_ns, ab)) { fail(2); return false; }
         tc_fence_after();
         const int st = i % kStages;
         const uint64_t pdesc = make_sdesc(p_base + (i & 1) * C::P_BYTES, 16, 1024, kSwizzle128);
@@ -242,15 +242,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mma_commit(&kv_empty[st]);
         return true;
       };
-      bool ok = mbar_wait(q_ready, 0, p.spin, ab);
+      bool ok = mbar_wait(q_ready, 0, p.wait_ns, ab);
       if (!ok) fail(3);
       tc_fence_after();
       for (int j = 0; j < nchunks && ok; ++j) {
         const int st = j % kStages;
         prog[1] = j;
-        if (!mbar_wait(&kv_full[st], (j / kStages) & 1, p.spin, ab)) { fail(4); ok = false; break; }
+        if (!mbar_wait(&kv_full[st], (j / kStages) & 1, p.wait_ns, ab)) { fail(4); ok = false; break; }
         fence_proxy_async_smem();
-        if (j >= 1 && !mbar_wait(&s_free[0], (j - 1) & 1, p.spin, ab)) { fail(5); ok = false; break; }
+        if (j >= 1 && !mbar_wait(&s_free[0], (j - 1) & 1, p.wait_ns, ab)) { fail(5); ok = false; break; }
         tc_fence_after();
         const uint32_t sbase = kv_base + st * C::STAGE_BYTES;
         for (int ks = 0; ks < nks; ++ks) {
@@ -264,7 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (ok && nchunks > 0) do_pv(nchunks - 1);
       mma_commit(mma_done);
-      mbar_wait(mma_done, 0, p.spin, no_abort);
+      mbar_wait(mma_done, 0, p.wait_ns, no_abort);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
@@ -296,8 +296,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int hs = h & 15;
     // every lane polls; the warp proceeds only if all lanes saw the phase
     auto wwait = [&](uint64_t* bar, uint32_t parity, bool cluster) -> bool {
-      const bool r = cluster ? mbar_wait_cluster(bar, parity, p.spin, ab)
-                             : mbar_wait(bar, parity, p.spin, ab);
+      const bool r = cluster ? mbar_wait_cluster(bar, parity, p.wait_ns, ab)
+                             : mbar_wait(bar, parity, p.wait_ns, ab);
       return __all_sync(0xffffffffu, r);
     };
     float m_used = -INFINITY, l = 0.f;
@@ -524,7 +524,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   p.nsplit = a.nsplit;
   p.kc = ((a.k + a.nsplit - 1) / a.nsplit + kN - 1) / kN * kN;
   p.scale_log2 = a.tau * 1.4426950408889634f;
-  p.spin = c.spin_limit;
+  p.wait_ns = c.wait_ns;
   p.err = c.err;
   const long long rows = (long long)a.B * a.T;
   p.part_o = a.part;

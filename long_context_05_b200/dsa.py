@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = [
     "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk",
     "dsa_sparse_attn", "dsa_forward", "dsa_prefill", "dsa_decode", "dsa_get_device_error",
-    "dsa_set_spin_limit", "dsa_launch_count",
+    "dsa_set_wait_timeout_us", "dsa_launch_count",
 ]
 
 
@@ -80,8 +80,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.dsa_launch_count.restype = ctypes.c_ulonglong
         L.dsa_launch_count.argtypes = []
-        L.dsa_set_spin_limit.restype = None
-        L.dsa_set_spin_limit.argtypes = [ctypes.c_longlong]
+        L.dsa_set_wait_timeout_us.restype = None
+        L.dsa_set_wait_timeout_us.argtypes = [ctypes.c_longlong]
         _lib = L
     return _lib
 
@@ -199,8 +199,8 @@ def launch_count() -> int:
     return int(lib().dsa_launch_count())
 
 
-def set_spin_limit(n: int) -> None:
-    lib().dsa_set_spin_limit(int(n))
+def set_wait_timeout_us(us: int) -> None:
+    lib().dsa_set_wait_timeout_us(int(us))
 
 
 @dataclass
