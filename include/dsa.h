@@ -180,6 +180,14 @@ DSA_API unsigned long long dsa_launch_count(void);
  * values <= 0 restore the default.  A small value is a test hook. */
 DSA_API void dsa_set_wait_timeout_us(long long microseconds);
 
+/* Failure-detection self test (no counterpart on the pages): launches one
+ * small kernel whose bounded wait can never be satisfied, so it gives up after
+ * the wait timeout (dsa_set_wait_timeout_us) and records DSA_ERR_TIMEOUT in
+ * the device error word, which the caller then reads with
+ * dsa_get_device_error().  Returns the launch status.  Nothing faults, traps
+ * or hangs. */
+DSA_API dsa_status dsa_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

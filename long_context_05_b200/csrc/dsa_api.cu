@@ -281,6 +281,13 @@ dsa_status dsa_decode(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, f
   return dsa_forward(&m, in, out, lse, idx_out, ws, ws_bytes, stream);
 }
 
+dsa_status dsa_selftest_wait_timeout(void* stream) {
+  LaunchCtx c;
+  dsa_status st = make_ctx(stream, &c);
+  if (st != DSA_OK) return st;
+  return from_cuda(launch_wait_timeout_probe(c));
+}
+
 dsa_status dsa_get_device_error(void* stream, int* detail) {
   if (detail) *detail = 0;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;

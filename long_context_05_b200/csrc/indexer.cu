@@ -315,8 +315,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < QPS; ++q) {
             const int t = it.t0 + j * QPS + q;
-            if (t < it.tend && s <= p.S - p.T + t)
-              p.scores[((size_t)it.b * p.q_count + (t - p.q_begin)) * p.ld + s] = accq[q] * ks;
+            if (t < it.tend && s <= p.S - p.T + t) {
+              // self-check: the score slot lies inside this launch's tile
+              const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
+              if (ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld)
+                p.scores[ri * p.ld + s] = accq[q] * ks;
+              else
+                report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
+            }
           }
         }
       }

@@ -81,6 +81,8 @@ size_t topk_workspace_bytes(int rows);
 bool topk_uses_workspace(int rows, int S, int num_sms);
 cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a);
 
+cudaError_t launch_wait_timeout_probe(const LaunchCtx& c);
+
 // split-k partial buffer size (floats) for a decode attention launch
 size_t attn_partial_floats(int rows, int H, int d_v, int nsplit);
 int attn_choose_nsplit(int rows, int H, int k, int num_sms);

@@ -89,6 +89,7 @@ struct AttnParams {
   float* part_o;    // [rows, nsplit, H, d_v] (split mode)
   float* part_lse;  // [rows, nsplit, H], log2 units
   int T, S, H, k;
+  int rows;         // B * T query rows
   int nsplit, kc;   // splits per row and selected slots per split
   float scale_log2; // tau * log2(e)
   long long wait_ns;
@@ -135,7 +136,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int b = row / p.T;
   const int slot0 = split * p.kc;
   const int slot1 = min(p.k, slot0 + p.kc);
-  const int nchunks = (slot1 - slot0 + kN - 1) / kN;
+  // self-check: a cluster outside the launch's rows does no work
+  const bool row_ok = row >= 0 && row < p.rows && split >= 0 && split < p.nsplit && slot0 >= 0;
+  const int nchunks = row_ok ? (slot1 - slot0 + kN - 1) / kN : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -202,9 +205,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (c16 == 0) sMeta[st * kN + r] = valid ? 1 : 0;
         const uint16_t* src = kvb + (size_t)(valid ? iv : 0) * DK;
         for (int a = atom_lo; a < atom_hi; ++a) {
-          if (a * 128 + c16 * 16 < DK * 2)
-            cp_async16(stage + (a - atom_lo) * C::ATOM_BYTES + r * 128 + ((c16 ^ (r & 7)) << 4),
-                       src + a * 64 + c16 * 8);
+          const int doff = (a - atom_lo) * C::ATOM_BYTES + r * 128 + ((c16 ^ (r & 7)) << 4);
+          if (a * 128 + c16 * 16 < DK * 2) {
+            if (doff >= 0 && doff + 16 <= C::STAGE_BYTES)  // self-check: inside the stage
+              cp_async16(stage + doff, src + a * 64 + c16 * 8);
+            else
+              report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (13u << 8));
+          }
         }
       }
       cp_async_commit();
@@ -457,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           p.part_lse[((size_t)row * p.nsplit + split) * p.H + h] = lse2;
         }
       }
-    } else if (ok && h < p.H) {
+    } else if (ok && h < p.H && row_ok) {
       // no selected slots in this split: empty result
       if (p.nsplit > 1 && rank == 0) p.part_lse[((size_t)row * p.nsplit + split) * p.H + h] = -INFINITY;
     }
@@ -521,6 +528,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   p.S = a.S;
   p.H = a.H;
   p.k = a.k;
+  p.rows = a.B * a.T;
   p.nsplit = a.nsplit;
   p.kc = ((a.k + a.nsplit - 1) / a.nsplit + kN - 1) / kN * kN;
   p.scale_log2 = a.tau * 1.4426950408889634f;

@@ -147,9 +147,23 @@ struct Smem {
 
 // Steps 2-3 on a row whose threshold bin B (and the count above it) is known.
 // keys_in_bin: number of keys in bin B over the whole row.
+// Self-check on every output slot: a position outside [0, k) is recorded as
+// DSA_ERR_DEVICE_BOUNDS (detail names the write site) and skipped.
+__device__ __forceinline__ void put(int32_t* out, int k, int pos, int value, DevErr* err, unsigned site) {
+  if (pos >= 0 && pos < k) {
+    out[pos] = value;
+  } else {
+    report_error(err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_TOPK | (site << 8));
+  }
+}
+
 __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, unsigned int B, unsigned int above,
-                                unsigned int keys_in_bin, Smem& sm) {
+                                unsigned int keys_in_bin, Smem& sm, DevErr* err) {
   const int tid = threadIdx.x;
+  if (B >= (unsigned)kBins || above >= (unsigned)k) {  // threshold bin must exist
+    if (tid == 0) report_error(err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_TOPK | (9u << 8));
+    return;
+  }
   const unsigned int need = (unsigned int)k - above;  // keys to take from bin B (>= 1)
   if (tid == 0) {
     sm.cnt = 0;
@@ -162,31 +176,35 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
     const unsigned int key = order_key(row[x]);
     const unsigned int bin = key >> kBinShift;
     if (bin > B) {
-      out[atomicAdd(&sm.cnt, 1)] = x;
+      put(out, k, atomicAdd(&sm.cnt, 1), x, err, 1);
     } else if (bin == B && fits) {
       const int p = atomicAdd(&sm.ncand, 1);
-      sm.ck[p] = key;
-      sm.ci[p] = x;
+      if (p < kCap) {
+        sm.ck[p] = key;
+        sm.ci[p] = x;
+      } else {
+        report_error(err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_TOPK | (7u << 8));
+      }
     }
   }
   __syncthreads();
   unsigned int thr, krem;
   if (fits) {
-    const int nc = sm.ncand;
+    const int nc = min(sm.ncand, kCap);
     const unsigned int* ck = sm.ck;
     thr = radix_select([ck](int i) { return ck[i]; }, nc, B << kBinShift, 0xFFFFFFFFu << kBinShift, kBinShift,
                        need, sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
     // candidates above thr
     unsigned int eq_local = 0;
     for (int i = tid; i < nc; i += kThreads) {
-      if (sm.ck[i] > thr) out[atomicAdd(&sm.cnt, 1)] = sm.ci[i];
+      if (sm.ck[i] > thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 2);
       eq_local += sm.ck[i] == thr;
     }
     block_scan(eq_local, sm.warp_tot, &sm.total);
     const unsigned int E = sm.total;
     if (E == krem) {
       for (int i = tid; i < nc; i += kThreads)
-        if (sm.ck[i] == thr) out[atomicAdd(&sm.cnt, 1)] = sm.ci[i];
+        if (sm.ck[i] == thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 3);
       return;
     }
     // more equal keys than slots: keep the lowest indices.  Gather the equal
@@ -194,15 +212,18 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
     if (tid == 0) sm.eq_base = 0;
     __syncthreads();
     for (int i = tid; i < nc; i += kThreads)
-      if (sm.ck[i] == thr) sm.eqi[atomicAdd(&sm.eq_base, 1)] = sm.ci[i];
+      if (sm.ck[i] == thr) {
+        const int p = atomicAdd(&sm.eq_base, 1);
+        if (p < kCap) sm.eqi[p] = sm.ci[i];
+      }
     __syncthreads();
-    const int ne = sm.eq_base;
+    const int ne = min(sm.eq_base, kCap);
     const int* ci = sm.eqi;
     unsigned int krem2;
     const unsigned int ithr = radix_select([ci](int i) { return ~(unsigned int)ci[i]; }, ne, 0u, 0u, 32, krem,
                                            sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem2);
     for (int i = tid; i < ne; i += kThreads)
-      if (~(unsigned int)sm.eqi[i] >= ithr) out[atomicAdd(&sm.cnt, 1)] = sm.eqi[i];
+      if (~(unsigned int)sm.eqi[i] >= ithr) put(out, k, atomicAdd(&sm.cnt, 1), sm.eqi[i], err, 4);
     return;
   }
   // bin B too large for shared memory: radix passes over the row itself
@@ -216,7 +237,7 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
     const int x = base + tid;
     const bool valid = x < n;
     const unsigned int key = valid ? order_key(row[x]) : 0u;
-    if (valid && (key >> kBinShift) == B && key > thr) out[atomicAdd(&sm.cnt, 1)] = x;
+    if (valid && (key >> kBinShift) == B && key > thr) put(out, k, atomicAdd(&sm.cnt, 1), x, err, 5);
     const bool eq = valid && key == thr;
     const unsigned int bal = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) sm.warp_eq[warp] = __popc(bal);
@@ -224,7 +245,7 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
     int before = sm.eq_base;
     for (int w = 0; w < warp; ++w) before += sm.warp_eq[w];
     before += __popc(bal & ((1u << lane) - 1u));
-    if (eq && before < (int)krem) out[atomicAdd(&sm.cnt, 1)] = x;
+    if (eq && before < (int)krem) put(out, k, atomicAdd(&sm.cnt, 1), x, err, 6);
     __syncthreads();
     if (tid == 0) {
       int tot = 0;
@@ -265,7 +286,7 @@ __device__ void histogram_pass(const float* row, int lo, int hi, unsigned int* h
 }
 
 // One block per row.
-__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(TopkArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(TopkArgs a, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   int b, t, n;
@@ -278,13 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(TopkArgs a) {
     return;
   }
   for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = 0u;
+  if (threadIdx.x == 0) sm.bin = 0xFFFFFFFFu;
   __syncthreads();
   histogram_pass(row, 0, n, sm.hist);
   __syncthreads();
   find_bin(sm.hist, kBins, (unsigned int)k, sm.warp_tot, &sm.bin, &sm.above, &sm.total);
-  const unsigned int B = sm.bin, above = sm.above, inbin = sm.hist[B];
+  const unsigned int B = sm.bin, above = sm.above;
+  const unsigned int inbin = B < (unsigned)kBins ? sm.hist[B] : 0u;
   __syncthreads();
-  select_from_bin(row, n, k, out, B, above, inbin, sm);
+  select_from_bin(row, n, k, out, B, above, inbin, sm, err);
 }
 
 // ---------------------------------------------------------------- split path
@@ -310,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, 
     if (hist[x]) atomicAdd(&gh[x], hist[x]);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_seg_select_kernel(TopkArgs a, unsigned int* ghist) {
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_select_kernel(TopkArgs a, unsigned int* ghist, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   int b, t, n;
@@ -324,11 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_select_kernel(TopkArgs a
   }
   unsigned int* gh = ghist + (size_t)blockIdx.x * kBins;
   for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = gh[x];
+  if (threadIdx.x == 0) sm.bin = 0xFFFFFFFFu;
   __syncthreads();
   find_bin(sm.hist, kBins, (unsigned int)k, sm.warp_tot, &sm.bin, &sm.above, &sm.total);
-  const unsigned int B = sm.bin, above = sm.above, inbin = sm.hist[B];
+  const unsigned int B = sm.bin, above = sm.above;
+  const unsigned int inbin = B < (unsigned)kBins ? sm.hist[B] : 0u;
   __syncthreads();
-  select_from_bin(row, n, k, out, B, above, inbin, sm);
+  select_from_bin(row, n, k, out, B, above, inbin, sm, err);
 }
 
 __global__ void topk_zero_kernel(unsigned int* p, size_t n) {
@@ -352,7 +377,7 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
   if (!split) {
     e = cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_row_kernel<<<rows, kThreads, smem, c.stream>>>(a);
+    topk_row_kernel<<<rows, kThreads, smem, c.stream>>>(a, c.err);
     note_launches(1);
     return cudaGetLastError();
   }
@@ -362,7 +387,7 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
   topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, gh);
   e = cudaFuncSetAttribute(topk_seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_seg_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, gh);
+  topk_seg_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, gh, c.err);
   note_launches(2);
   return cudaGetLastError();
 }

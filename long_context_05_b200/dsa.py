@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = [
     "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk",
     "dsa_sparse_attn", "dsa_forward", "dsa_prefill", "dsa_decode", "dsa_get_device_error",
-    "dsa_set_wait_timeout_us", "dsa_launch_count",
+    "dsa_set_wait_timeout_us", "dsa_launch_count", "dsa_selftest_wait_timeout",
 ]
 
 
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.dsa_launch_count.restype = ctypes.c_ulonglong
         L.dsa_launch_count.argtypes = []
+        L.dsa_selftest_wait_timeout.restype = i
+        L.dsa_selftest_wait_timeout.argtypes = [vp]
         L.dsa_set_wait_timeout_us.restype = None
         L.dsa_set_wait_timeout_us.argtypes = [ctypes.c_longlong]
         _lib = L
@@ -197,6 +199,10 @@ def device_error() -> tuple[int, int]:
 
 def launch_count() -> int:
     return int(lib().dsa_launch_count())
+
+
+def selftest_wait_timeout() -> None:
+    _check("dsa_selftest_wait_timeout", lib().dsa_selftest_wait_timeout(_stream()))
 
 
 def set_wait_timeout_us(us: int) -> None:

@@ -227,3 +227,24 @@ def test_out_of_range_index_is_reported_not_read():
     st, det = dsa.device_error()
     assert st == 6 and (det & 0xF0) == 0x30
     assert dsa.device_error()[0] == 0   # cleared by the read
+
+
+def test_bounded_wait_reports_timeout():
+    """A wait that can never be satisfied gives up after the configured limit
+    and reports DSA_ERR_TIMEOUT; the context stays usable afterwards."""
+    import time
+    dsa.set_wait_timeout_us(20000)            # 20 ms
+    try:
+        t0 = time.perf_counter()
+        dsa.selftest_wait_timeout()
+        st, det = dsa.device_error()
+        dt = time.perf_counter() - t0
+    finally:
+        dsa.set_wait_timeout_us(0)           # back to the default
+    assert st == 5 and (det & 0xFF) == 0x50
+    assert dt < 5.0
+    assert dsa.device_error()[0] == 0
+    # the library still works after the timeout
+    wl = WORKLOADS["tiny_prefill_256"]
+    inp = {k: v.cuda() for k, v in make_inputs(wl, "cpu").items()}
+    _run_forward(wl, inp)
