@@ -132,6 +132,29 @@ DSA_API dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
                     int64_t ld_scores, int q_begin, int q_count, int32_t* idx,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* Step B without any allocation (an addition of this library; the sparse
+ * attention papers have no counterpart).  Same arguments, output and error
+ * checks as dsa_topk, minus the workspace: the per-row histograms of the split
+ * top-k path live in a fixed array of DSA_TOPK_STATIC_MAX_ROWS x 2048 words
+ * (512 KiB) compiled into the library, so neither this call nor anything it
+ * calls allocates memory.  It is meant for callers that cannot allocate at
+ * call time: a C host program given only the score and index buffers, or a
+ * decode loop whose HBM is reserved up front for weights and the key cache,
+ * where a late cudaMalloc could fail or synchronise the device.
+ *   - B * q_count > DSA_TOPK_STATIC_MAX_ROWS: DSA_ERR_WORKSPACE, nothing
+ *     launched (use dsa_topk for more rows);
+ *   - each call first clears the histogram rows it uses, in stream order;
+ *   - all calls on a device share the array: calls whose launches may run at
+ *     the same time on the GPU (unordered streams, concurrent host threads)
+ *     race on it and may return wrong indices; calls in sequence on one
+ *     stream are safe;
+ *   - the first call on a device looks up the array's address with that device
+ *     current; make that first call before any stream capture begins. */
+#define DSA_TOPK_STATIC_MAX_ROWS 64
+DSA_API dsa_status dsa_topk_static(const dsa_shape* shape, const float* scores,
+                           int64_t ld_scores, int q_begin, int q_count,
+                           int32_t* idx, void* stream);
+
 /* Step C -- sparse MQA/MLA attention over the selected keys.
  *   q   [B, T, H, d_k] BF16;  kv [B, S, d_k] BF16 (V = kv[..., :d_v]);
  *   idx [B, T, k] int32, -1 = empty slot (skipped), duplicates counted twice;

@@ -161,6 +161,10 @@ bool indexer_ptrs_ok(const uint8_t* q_I, const float* q_scale, const float* w, c
 }
 
 }  // namespace
+
+dsa_status api_check_shape(const dsa_shape* s) { return check_shape(s); }
+dsa_status api_make_ctx(void* stream, LaunchCtx* c) { return make_ctx(stream, c); }
+
 }  // namespace dsa
 
 using namespace dsa;

@@ -78,10 +78,17 @@ cudaError_t launch_indexer(const LaunchCtx& c, const IndexerArgs& a);
 // ws: optional scratch for the split path (few long rows); see topk.cu
 cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t ws_bytes);
 size_t topk_workspace_bytes(int rows);
+// top-k split path into an explicit histogram array of rows * 2048 words
+cudaError_t launch_topk_split_into(const LaunchCtx& c, const TopkArgs& a, unsigned int* hist);
+constexpr int kTopkHistBins = 2048;
 bool topk_uses_workspace(int rows, int S, int num_sms);
 cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a);
 
 cudaError_t launch_wait_timeout_probe(const LaunchCtx& c);
+
+// shape validation and launch context of the public entry points (dsa_api.cu)
+dsa_status api_check_shape(const dsa_shape* s);
+dsa_status api_make_ctx(void* stream, LaunchCtx* c);
 
 // split-k partial buffer size (floats) for a decode attention launch
 size_t attn_partial_floats(int rows, int H, int d_v, int nsplit);

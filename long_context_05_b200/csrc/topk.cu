@@ -393,3 +393,22 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
 }
 
 }  // namespace dsa
+
+namespace dsa {
+
+// Split path with a caller-provided histogram array (B * q_count * 2048
+// words): zero it, histogram each row over several blocks, select per row.
+cudaError_t launch_topk_split_into(const LaunchCtx& c, const TopkArgs& a, unsigned int* hist) {
+  const int rows = a.B * a.q_count;
+  if (rows <= 0) return cudaSuccess;
+  topk_zero_kernel<<<64, 256, 0, c.stream>>>(hist, (size_t)rows * kBins);
+  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, hist);
+  const size_t smem = sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_seg_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, hist, c.err);
+  note_launches(3);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

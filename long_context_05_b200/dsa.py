@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = [
     "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk",
     "dsa_sparse_attn", "dsa_forward", "dsa_prefill", "dsa_decode", "dsa_get_device_error",
-    "dsa_set_wait_timeout_us", "dsa_launch_count", "dsa_selftest_wait_timeout",
+    "dsa_set_wait_timeout_us", "dsa_launch_count", "dsa_selftest_wait_timeout", "dsa_topk_static",
 ]
 
 
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_scores.argtypes = [sp, vp, vp, vp, vp, vp, i, i, vp, i64, vp]
         L.dsa_topk.restype = i
         L.dsa_topk.argtypes = [sp, vp, i64, i, i, vp, vp, sz, vp]
+        L.dsa_topk_static.restype = i
+        L.dsa_topk_static.argtypes = [sp, vp, i64, i, i, vp, vp]
         L.dsa_sparse_attn.restype = i
         L.dsa_sparse_attn.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
         for fn in ("dsa_forward", "dsa_prefill", "dsa_decode"):
@@ -153,6 +155,16 @@ def topk(shape: Shape, scores: torch.Tensor, q_begin: int, q_count: int, idx: to
     _check("dsa_topk", lib().dsa_topk(
         ctypes.byref(shape), _p(scores), scores.shape[-1], q_begin, q_count, _p(idx),
         _p(ws), 0 if ws is None else ws.numel(), _stream()))
+    return idx
+
+
+def topk_static(shape: Shape, scores: torch.Tensor, q_begin: int, q_count: int,
+                idx: torch.Tensor) -> torch.Tensor:
+    """Step B with the library's fixed histogram array (no workspace, no allocation)."""
+    _need(scores, torch.float32, "scores")
+    _need(idx, torch.int32, "idx")
+    _check("dsa_topk_static", lib().dsa_topk_static(
+        ctypes.byref(shape), _p(scores), scores.shape[-1], q_begin, q_count, _p(idx), _stream()))
     return idx
 
 
