@@ -283,9 +283,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kNSub;
           const float* wq = wbuf + j * kNSub;
-          float accq[QPS];
+          // w * ReLU(x) summed over the heads of each query: four independent
+          // packed-pair partial sums per query keep the FMA chains short
+          constexpr int NP = HI >= 8 ? 4 : 2;
+          float2 part[QPS][NP];
 #pragma unroll
-          for (int q = 0; q < QPS; ++q) accq[q] = 0.f;
+          for (int q = 0; q < QPS; ++q)
+#pragma unroll
+            for (int i = 0; i < NP; ++i) part[q][i] = make_float2(0.f, 0.f);
           uint32_t v[2][32];
           tmem_ld32(taddr, v[0]);
           tmem_wait_ld_dep(v[0]);
@@ -300,17 +305,27 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lane == 0) mbar_arrive(&acc_empty[acc]);
             }
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 w4 = *reinterpret_cast<const float4*>(wq + c * 32 + e);
+            for (int e = 0; e < 32; e += 2 * NP) {
               const int q = (c * 32 + e) / HI;
-              float a = accq[q];
-              a = fmaf(w4.x, fmaxf(__uint_as_float(v[c & 1][e + 0]), 0.f), a);
-              a = fmaf(w4.y, fmaxf(__uint_as_float(v[c & 1][e + 1]), 0.f), a);
-              a = fmaf(w4.z, fmaxf(__uint_as_float(v[c & 1][e + 2]), 0.f), a);
-              a = fmaf(w4.w, fmaxf(__uint_as_float(v[c & 1][e + 3]), 0.f), a);
-              accq[q] = a;
+#pragma unroll
+              for (int i = 0; i < NP; i += 2) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wq + c * 32 + e + 2 * i);
+                const uint32_t* x = &v[c & 1][e + 2 * i];
+                const float2 r0 = make_float2(fmaxf(__uint_as_float(x[0]), 0.f), fmaxf(__uint_as_float(x[1]), 0.f));
+                const float2 r1 = make_float2(fmaxf(__uint_as_float(x[2]), 0.f), fmaxf(__uint_as_float(x[3]), 0.f));
+                part[q][i] = __ffma2_rn(make_float2(w4.x, w4.y), r0, part[q][i]);
+                part[q][i + 1] = __ffma2_rn(make_float2(w4.z, w4.w), r1, part[q][i + 1]);
+              }
             }
             if (c + 1 < kNSub / 32) tmem_wait_ld_dep(v[(c + 1) & 1]);
+          }
+          float accq[QPS];
+#pragma unroll
+          for (int q = 0; q < QPS; ++q) {
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < NP; ++i) a += part[q][i].x + part[q][i].y;
+            accq[q] = a;
           }
 #pragma unroll
           for (int q = 0; q < QPS; ++q) {

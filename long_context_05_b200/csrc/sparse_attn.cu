@@ -172,20 +172,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t* irow = p.idx + (size_t)row * p.k;
     const uint16_t* kvb = p.kv + (size_t)b * p.S * DK;
     uint8_t* stage = sKV + w * C::STAGE;
+    // the indices of a chunk are loaded one chunk ahead, while the previous
+    // chunk's rows are in flight
+    int ivn[kN / 4];
+    auto load_idx = [&](int j) {
+#pragma unroll
+      for (int m = 0; m < kN / 4; ++m) {
+        const int slot = slot0 + j * kN + rg + 4 * m;
+        ivn[m] = (j < nchunks && slot < slot1) ? irow[slot] : -1;
+      }
+    };
+    load_idx(w);
     for (int j = w, use = 0; j < nchunks; j += kStages, ++use) {
+      int iv[kN / 4];
+#pragma unroll
+      for (int m = 0; m < kN / 4; ++m) iv[m] = ivn[m];
       if (!mbar_wait(&kv_empty[w], (use & 1) ^ 1, p.wait_ns, ab)) { fail(1); break; }
 #pragma unroll
       for (int m = 0; m < kN / 4; ++m) {
         const int r = rg + 4 * m;
-        const int slot = slot0 + j * kN + r;
-        int iv = slot < slot1 ? irow[slot] : -1;
-        if (iv >= p.S) {
+        int v = iv[m];
+        if (v >= p.S) {
           if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
-          iv = -1;
+          v = -1;
         }
-        const bool valid = iv >= 0;
+        const bool valid = v >= 0;
         if (c16 == 0) sMeta[w * kN + r] = valid ? 1 : 0;
-        const uint16_t* src = kvb + (size_t)(valid ? iv : 0) * DK;
+        const uint16_t* src = kvb + (size_t)(valid ? v : 0) * DK;
 #pragma unroll
         for (int a = 0; a < C::NATOM; ++a) {
           if (a * 128 + c16 * 16 < DK * 2)
@@ -193,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       cp_async_commit();
+      load_idx(j + kStages);
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(&kv_full[w]);
@@ -208,8 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(sQ), kv_base = smem_u32(sKV), p_base = smem_u32(sP);
       const uint32_t v_atom = (uint32_t)(half * C::DVH / 64);
       int pv_issued = 0;
-      auto do_pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1, p.wait_ns, ab)) { fail(2); return false; }
+      auto issue_pv = [&](int i) {
         tc_fence_after();
         const int st = i & 1;
         const uint32_t vbase = kv_base + st * C::STAGE + v_atom * C::KV_ATOM;
@@ -222,29 +235,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(pv_done);
         mma_commit(&kv_empty[st]);
         pv_issued = i + 1;
-        return true;
       };
       bool ok = nchunks == 0 || mbar_wait(q_full, 0, p.wait_ns, ab);
       if (!ok) fail(3);
-      for (int j = 0; j < nchunks && ok; ++j) {
-        const int st = j & 1, sb = j & 1;
-        if (!mbar_wait(&kv_full[st], (j >> 1) & 1, p.wait_ns, ab)) { fail(4); ok = false; break; }
-        fence_proxy_async_smem();
-        if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, p.wait_ns, ab)) { fail(5); ok = false; break; }
-        tc_fence_after();
-        const uint32_t sbase = kv_base + st * C::STAGE;
+      // Issue whichever MMA is ready: Q K^T of chunk qk once its rows have
+      // landed (and its S buffer is free), P V of chunk pv once its
+      // probabilities are written.  P V never waits behind a later chunk's
+      // gather, so a stage is handed back to its gather warp as early as the
+      // data dependencies allow.
+      int qk = 0, pv = 0;
+      uint64_t t_idle = 0;
+      uint32_t spins = 0;
+      while (ok && pv < nchunks) {
+        bool progressed = false;
+        if (qk < nchunks && qk <= pv + 1) {
+          const int st = qk & 1;
+          if (mbar_test_wait(&kv_full[st], (qk >> 1) & 1) &&
+              (qk < 2 || mbar_test_wait(&s_free[st], ((qk >> 1) - 1) & 1))) {
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const uint32_t sbase = kv_base + st * C::STAGE;
 #pragma unroll 4
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const int d = ks * 16;
-          const uint32_t off = (uint32_t)((d % 64) * 2);
-          const uint64_t adesc = make_sdesc(q_base + (d / 64) * C::Q_ATOM + off, 16, 1024, kSwizzle128);
-          const uint64_t bdesc = make_sdesc(sbase + (d / 64) * C::KV_ATOM + off, 16, 1024, kSwizzle128);
-          mma_bf16(tmem + kSCol + sb * kN, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < C::KSTEPS; ++ks) {
+              const int d = ks * 16;
+              const uint32_t off = (uint32_t)((d % 64) * 2);
+              const uint64_t adesc = make_sdesc(q_base + (d / 64) * C::Q_ATOM + off, 16, 1024, kSwizzle128);
+              const uint64_t bdesc = make_sdesc(sbase + (d / 64) * C::KV_ATOM + off, 16, 1024, kSwizzle128);
+              mma_bf16(tmem + kSCol + st * kN, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&s_full[st]);
+            ++qk;
+            progressed = true;
+          }
         }
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !do_pv(j - 1)) { ok = false; break; }
+        if (pv < qk && mbar_test_wait(p_full, pv & 1)) {
+          issue_pv(pv);
+          ++pv;
+          progressed = true;
+        }
+        if (progressed) {
+          spins = 0;
+          continue;
+        }
+        // nothing ready: doze briefly on the event most likely next, with
+        // bounded idle time, and abort when another role failed
+        if (pv < qk)
+          mbar_try_wait_hint(p_full, pv & 1, 200);
+        else
+          mbar_try_wait_hint(&kv_full[qk & 1], (qk >> 1) & 1, 200);
+        if (++spins == 1) t_idle = global_ns();
+        if ((spins & 1023u) == 0u) {
+          if (*abort_flag != 0) { ok = false; break; }
+          const long long dt = (long long)(global_ns() - t_idle);
+          if (dt > p.wait_ns || (dt > 1000000 && (spins & 65535u) == 0u && p.err->code != 0u)) {
+            fail(4);
+            ok = false;
+          }
+        }
       }
-      if (ok && nchunks > 0) do_pv(nchunks - 1);
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
       // drain: the last releases of each stage are never waited by the gather
