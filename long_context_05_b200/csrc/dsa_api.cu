@@ -113,7 +113,7 @@ WsLayout ws_layout(const dsa_shape* s, int num_sms) {
   L.q_rows = s->mode == DSA_DECODE ? s->T : q_block_of(s);
   L.scores_off = 0;
   L.scores_bytes = round_up((size_t)s->B * L.q_rows * scores_ld(s) * sizeof(float), 256);
-  L.nsplit = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->k, num_sms) : 1;
+  L.nsplit = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->d_v, s->k, num_sms) : 1;
   L.part_off = L.scores_off + L.scores_bytes;
   L.part_bytes = round_up(attn_partial_floats(s->B * s->T, s->H, s->d_v, L.nsplit) * sizeof(float), 256);
   L.topk_off = L.part_off + L.part_bytes;

@@ -17,11 +17,12 @@
 // sub-tiles, so each byte of k_I fetched serves 8 MMAs.  Tiles entirely
 // above the causal diagonal are skipped.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over the work items):
+// Warp roles (448 threads, one CTA per SM, persistent over the work items):
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..9  epilogue: two groups of four warps (one per TMEM lane
-//               quarter); group g drains accumulators u with u % 2 == g
+//   warps 2..13 epilogue: three groups of four warps (one per TMEM lane
+//               quarter); group g drains sub-tiles u with u % 3 == g, so
+//               three warps per SM sub-partition hide each other's latency
 // Four TMEM accumulators of 128 columns each let the MMA run up to three
 // sub-tiles ahead of the epilogue.
 #include "internal.h"
@@ -36,11 +37,12 @@ using namespace sm100;
 constexpr int kBM = 128;       // keys per tile (MMA M)
 constexpr int kNSub = 128;     // MMA N: (query, head) rows per sub-tile
 constexpr int kMaxNB = 8;      // sub-tiles per work item
-constexpr int kKC = 32;        // key tiles per work item
+constexpr int kKC = 32;        // key tiles per work item (at most; fewer when items are scarce)
 constexpr int kStages = 4;     // depth of the k_I ring
 constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * kNSub = 512 columns)
-constexpr int kThreads = 320;
-constexpr int kEpiThreads = 256;
+constexpr int kEpiGroups = 3;   // epilogue groups of four warps
+constexpr int kEpiThreads = 128 * kEpiGroups;
+constexpr int kThreads = 64 + kEpiThreads;
 
 struct IdxParams {
   const float* w;
@@ -50,6 +52,7 @@ struct IdxParams {
   long long ld;
   int B, T, S, q_begin, q_count;
   int nb;              // B sub-tiles per item
+  int kc;              // key tiles per item
   int groups_per_seq;  // query groups per sequence
   long long wait_ns;
   DevErr* err;
@@ -94,7 +97,7 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
     it.tend = min(it.t0 + per_group, q_end);
     const int pos_last = p.S - p.T + it.tend - 1;
     it.ntiles = pos_last / kBM + 1;
-    const int nch = (it.ntiles + kKC - 1) / kKC;
+    const int nch = (it.ntiles + p.kc - 1) / p.kc;
     int c0 = (int)(((long long)cta - flat) % grid);
     if (c0 < 0) c0 += grid;
     for (int c = c0; c < nch; c += grid) {
@@ -192,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nsub; ++j)
           tma_load_2d(sB + j * L::kBSubBytes, &tm_q, b_full, 0, (it.b * p.T + it.t0 + j * QPS) * HI);
         ++items;
-        const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
+        const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
           if (!mbar_wait(&a_empty[st], ((a_cnt / kStages) & 1) ^ 1, p.wait_ns, ab)) {
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for_each_item<HI>(p, [&](const Item& it) {
         if (!mbar_wait(b_full, items & 1, p.wait_ns, ab)) { fail(3); return false; }
         ++items;
-        const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
+        const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
           if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.wait_ns, ab)) { fail(4); return false; }
@@ -248,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    const int ew = warp - 2;             // 0..7
-    const int grp = ew >> 2;             // accumulator parity this warp drains
+    const int ew = warp - 2;             // 0 .. 4 * kEpiGroups - 1
+    const int grp = ew >> 2;             // drains sub-tiles u with u % kEpiGroups == grp
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;   // key row within the tile
     const int etid = threadIdx.x - 64;   // 0..255
@@ -269,14 +272,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&w_ready[items & 1]);
       if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.wait_ns, ab)) { fail(7); return false; }
       ++items;
-      const int kt0 = it.c * kKC, kt1 = min(kt0 + kKC, it.ntiles);
+      const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
       for (int kt = kt0; kt < kt1; ++kt) {
         const int s = kt * kBM + r;
         const float ks = s < p.S ? p.k_scale[(size_t)it.b * p.S + s] : 0.f;
         for (int j = 0; j < p.nb; ++j) {
           if (!subtile_active<HI>(p, it, j, kt)) continue;
           const uint32_t my = u++;
-          if ((int)(my & 1) != grp) continue;
+          if ((int)(my % kEpiGroups) != grp) continue;
           const int acc = my % kNAcc;
           const bool got = mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.wait_ns, ab);
           if (!__all_sync(0xffffffffu, got)) { fail(6); return false; }
@@ -382,15 +385,24 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   p.groups_per_seq = (a.q_count + per_group - 1) / per_group;
   p.wait_ns = c.wait_ns;
   p.err = c.err;
-  // count the items to size the grid
-  long long items = 0;
-  for (int g = 0; g < p.groups_per_seq; ++g) {
-    const int t0 = a.q_begin + g * per_group;
-    const int tend = t0 + per_group < a.q_begin + a.q_count ? t0 + per_group : a.q_begin + a.q_count;
-    const int ntiles = (a.S - a.T + tend - 1) / kBM + 1;
-    items += (ntiles + kKC - 1) / kKC;
+  // count the items to size the grid; with few query groups (decode) use
+  // shorter key runs so that every SM gets several items
+  auto count_items = [&](int kc) {
+    long long n = 0;
+    for (int g = 0; g < p.groups_per_seq; ++g) {
+      const int t0 = a.q_begin + g * per_group;
+      const int tend = t0 + per_group < a.q_begin + a.q_count ? t0 + per_group : a.q_begin + a.q_count;
+      const int ntiles = (a.S - a.T + tend - 1) / kBM + 1;
+      n += (ntiles + kc - 1) / kc;
+    }
+    return n * a.B;
+  };
+  p.kc = kKC;
+  long long items = count_items(p.kc);
+  while (p.kc > 4 && items < 4LL * c.num_sms) {
+    p.kc /= 2;
+    items = count_items(p.kc);
   }
-  items *= a.B;
   const int grid = (int)(items < c.num_sms ? items : c.num_sms);
   if (grid <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<DI, HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,

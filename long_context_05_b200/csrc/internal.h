@@ -92,6 +92,6 @@ dsa_status api_make_ctx(void* stream, LaunchCtx* c);
 
 // split-k partial buffer size (floats) for a decode attention launch
 size_t attn_partial_floats(int rows, int H, int d_v, int nsplit);
-int attn_choose_nsplit(int rows, int H, int k, int num_sms);
+int attn_choose_nsplit(int rows, int H, int d_v, int k, int num_sms);
 
 }  // namespace dsa

@@ -13,22 +13,29 @@
 // one per half of the value columns; each computes the full logit tile
 // (Q K^T over the 576-wide key) and its 128 x 256 half of the output.
 //
-// Per CTA: Q (128 x 576 BF16, 144 KB) is loaded once by TMA into shared
-// memory (128B swizzle); selected KV rows arrive in chunks of 32 through a
-// 2-stage ring filled with 16-byte cp.async by two gather warps that take
-// alternate chunks; both MMAs read their operands from shared memory
-// (S = Q K^T into a double-buffered TMEM tile, O += P V with P written by the
-// softmax warps in a 64B-swizzled tile and V read as the MN-major view of the
-// same gathered rows).  Online softmax in base 2 with a lazy rescale: the
-// running maximum moves only when a chunk exceeds it by more than 8 (so
-// p <= 256), and then the TMEM accumulator is rescaled once.
+// Per CTA:
+//   * TMEM: O (128 x 256 FP32) | two 32-column S buffers | the first 384
+//     columns of Q as BF16 pairs (192 columns) = 512 columns.  The rest of Q
+//     (192 columns, 48 KB) sits in shared memory, loaded once by TMA.  Q K^T
+//     takes its A operand from TMEM for 24 of its 36 K steps, which keeps
+//     those steps off the shared-memory port;
+//   * the rest of shared memory is a 4-stage ring of gathered key rows (32
+//     keys x 1152 B per stage), filled with 16-byte cp.async by one gather
+//     warp that keeps three chunks in flight;
+//   * the softmax writes the BF16 probabilities over the first half of the
+//     chunk's S buffer, and O += P V takes P from TMEM and V as the MN-major
+//     view of the gathered rows.  With two S/P buffers the softmax of chunk
+//     j+1 runs while P V of chunk j executes.
+// Online softmax in base 2 with a lazy rescale: the running maximum moves
+// only when a chunk exceeds it by more than 8 (so p <= 256), and then the
+// TMEM accumulator is rescaled once, after the previous P V has landed.
 //
-// Warp roles (224 threads): warps 0-1 gather (warp w fills stage w), warp 2
-// owns TMEM and issues the MMAs, warps 3-6 run the softmax (thread = head
-// row) and write the output.  Decode splits the selected keys of each query
-// over several CTAs and merges the partial results with a combine kernel.
-// Every barrier that receives an asynchronous arrival is waited on before
-// the CTA exits.
+// Warp roles (192 threads): warp 0 gathers, warp 1 owns TMEM and issues the
+// MMAs (whichever is ready: Q K^T of the next chunk or P V of the oldest),
+// warps 2-5 run the softmax (thread = head row) and write the output.
+// Decode splits the selected keys of each query over several CTAs and merges
+// the partial results with a combine kernel.  Every barrier that receives an
+// asynchronous arrival is waited on before the CTA exits.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -40,39 +47,49 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kN = 32;          // selected keys per chunk
-constexpr int kStages = 2;      // one per gather warp
-constexpr int kThreads = 224;
-constexpr int kMmaWarp = 2;
-constexpr uint32_t kOCol = 0, kSCol = 256, kTmemCols = 512;  // S: two buffers of kN columns
-constexpr float kRescaleThreshold = 8.f;                     // log2 units
+constexpr int kN = 32;          // selected keys per chunk (N of Q K^T)
+constexpr int kStages = 4;      // gather ring
+constexpr int kInFlight = 3;    // chunks the gather warp keeps in flight
+constexpr int kSBuf = 2;        // S/P buffers in TMEM
+constexpr int kThreads = 192;
+constexpr int kGatherWarp = 0, kMmaWarp = 1;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.f;  // log2 units
 
 template <int DK, int DV>
 struct Cfg {
-  static constexpr int KSTEPS = DK / 16;            // 16-wide MMA K steps over the key dim
-  static constexpr int NATOM = (DK + 63) / 64;      // 64-column (128-byte) atoms of a row
-  static constexpr bool SPLIT_V = DV >= 128;        // value columns split over two CTAs
-  static constexpr int NHALF = SPLIT_V ? 2 : 1;
+  static constexpr int KSTEPS = DK / 16;             // 16-wide MMA K steps over the key dim
+  static constexpr int NATOM = (DK + 63) / 64;       // 64-column (128-byte) atoms of a row
+  static constexpr int NHALF = DV >= 128 ? 2 : 1;    // value columns split over CTAs
   static constexpr int DVH = DV / NHALF;
-  static constexpr int Q_ATOM = 128 * 128;          // 128 head rows x 128 bytes
-  static constexpr int KV_ATOM = kN * 128;          // kN key rows x 128 bytes
+  static constexpr uint32_t OCOL = 0;
+  static constexpr uint32_t SCOL = (DVH + 31) / 32 * 32;
+  static constexpr uint32_t QCOL = SCOL + kSBuf * kN;
+  // leading key dims whose Q lives in TMEM (whole 64-wide atoms, or all of DK)
+  static constexpr int QT_FIT = (int)(kTmemCols - QCOL) * 2 / 64 * 64;
+  static constexpr int QT_DIMS = DK <= QT_FIT ? DK : QT_FIT;
+  static constexpr int QT_STEPS = QT_DIMS / 16;
+  static constexpr int QT_BLOCKS = (QT_DIMS + 63) / 64;  // 32-column stores per row
+  static constexpr int QS_ATOMS = (DK - QT_DIMS) / 64;   // Q atoms in shared memory
+  static constexpr int Q_ATOM = 128 * 128;               // 128 head rows x 128 bytes
+  static constexpr int KV_ATOM = kN * 128;               // kN key rows x 128 bytes
   static constexpr int STAGE = NATOM * KV_ATOM;
-  static constexpr int P_BYTES = 128 * kN * 2;      // 128 rows x 64 bytes, 64B swizzle
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + NATOM * Q_ATOM;
-  static constexpr int OFF_P = OFF_KV + kStages * STAGE;
-  static constexpr int OFF_META = OFF_P + P_BYTES;  // valid flag per slot, kStages x kN bytes
-  static constexpr int OFF_BAR = OFF_META + kStages * kN;
-  static constexpr int NBARS = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 1;
+  static constexpr int OFF_KV = OFF_Q + QS_ATOMS * Q_ATOM;
+  static constexpr int OFF_MASK = OFF_KV + kStages * STAGE;  // valid-slot bit mask per stage
+  static constexpr int OFF_BAR = OFF_MASK + kStages * 4;
+  static constexpr int NBARS = 2 + 2 * kStages + 3 * kSBuf + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
-  static_assert(DVH <= 256 && DVH % 16 == 0, "value columns per CTA");
-  static_assert(kSCol + 2 * kN <= kTmemCols && DVH <= kSCol, "TMEM layout");
+  static constexpr int ALLOC = BYTES + 1024;          // room to align the base to 1024
+  static_assert(DK % 64 == 0 || QT_DIMS == DK, "Q split on whole atoms");
+  static_assert(QT_DIMS % 16 == 0 && DVH <= 256 && DVH % 16 == 0, "shape");
+  static_assert(QCOL + (QT_DIMS / 2 + 31) / 32 * 32 <= kTmemCols, "TMEM layout");
   static_assert(ALLOC <= 232448, "shared memory per CTA");
 };
 
 struct AttnParams {
+  const uint16_t* q;
   const uint16_t* kv;
   const int32_t* idx;
   uint16_t* out;
@@ -92,6 +109,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// cp.async.wait_group with a run-time count (0 .. kInFlight - 1)
+__device__ __forceinline__ void cp_async_wait_upto(int n) {
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    default: cp_async_wait<2>(); break;
+  }
+}
+static_assert(kInFlight - 1 <= 2, "cp_async_wait_upto range");
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
@@ -100,17 +127,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sKV = smem + C::OFF_KV;
-  uint8_t* sP = smem + C::OFF_P;
-  uint8_t* sMeta = smem + C::OFF_META;
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;                // [kStages]
-  uint64_t* kv_empty = kv_full + kStages;      // [kStages]
-  uint64_t* s_full = kv_empty + kStages;       // [2]
-  uint64_t* s_free = s_full + 2;               // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* mma_done = pv_done + 1;
+  uint64_t* q_full = bars;                     // Q atoms in shared memory (TMA)
+  uint64_t* q_ready = q_full + 1;              // Q rows in TMEM (4 softmax warps)
+  uint64_t* kv_full = q_ready + 1;             // [kStages] rows landed (32 gather lanes)
+  uint64_t* kv_empty = kv_full + kStages;      // [kStages] stage consumed (MMA commit)
+  uint64_t* s_full = kv_empty + kStages;       // [kSBuf] S written (MMA commit)
+  uint64_t* p_full = s_full + kSBuf;           // [kSBuf] P written (4 softmax warps)
+  uint64_t* pv_done = p_full + kSBuf;          // [kSBuf] P V of the buffer complete (MMA commit)
+  uint64_t* mma_done = pv_done + kSBuf;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -128,16 +154,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_ready, 4);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&kv_full[i], 32);  // the 32 lanes of the gather warp that owns the stage
+      mbar_init(&kv_full[i], 32);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -157,23 +183,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     report_error(p.err, DSA_ERR_TIMEOUT, ERR_SITE_ATTN | (where << 8));
     *abort_flag = 1;
   };
+  // every lane polls; the warp proceeds only if all lanes saw the phase
+  auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const bool r = mbar_wait(bar, parity, p.wait_ns, ab);
+    return __all_sync(0xffffffffu, r);
+  };
 
-  if (warp < 2) {
-    // ------------------------------------------------------------ gather (warp w fills stage w)
-    const int w = warp;
+  if (warp == kGatherWarp) {
+    // ------------------------------------------------------------ gather
     bool q_issued = false;
-    if (w == 0 && lane == 0 && nchunks > 0) {
+    if (lane == 0 && nchunks > 0 && C::QS_ATOMS > 0) {
       prefetch_tmap(&tm_q);
-      mbar_arrive_expect_tx(q_full, C::NATOM * C::Q_ATOM);
-      for (int a = 0; a < C::NATOM; ++a) tma_load_2d(sQ + a * C::Q_ATOM, &tm_q, q_full, a * 64, row * p.H);
+      mbar_arrive_expect_tx(q_full, C::QS_ATOMS * C::Q_ATOM);
+      for (int a = 0; a < C::QS_ATOMS; ++a)
+        tma_load_2d(sQ + a * C::Q_ATOM, &tm_q, q_full, C::QT_DIMS + a * 64, row * p.H);
       q_issued = true;
     }
     const int c16 = lane & 7, rg = lane >> 3;  // 16-byte column chunk, row group
     const int32_t* irow = p.idx + (size_t)row * p.k;
     const uint16_t* kvb = p.kv + (size_t)b * p.S * DK;
-    uint8_t* stage = sKV + w * C::STAGE;
-    // the indices of a chunk are loaded one chunk ahead, while the previous
-    // chunk's rows are in flight
+    // indices are loaded one chunk ahead, while earlier rows are in flight
     int ivn[kN / 4];
     auto load_idx = [&](int j) {
 #pragma unroll
@@ -182,12 +211,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         ivn[m] = (j < nchunks && slot < slot1) ? irow[slot] : -1;
       }
     };
-    load_idx(w);
-    for (int j = w, use = 0; j < nchunks; j += kStages, ++use) {
+    int issued = 0, signaled = 0;
+    // wait until at most `keep` chunks are pending, then publish the others
+    auto retire = [&](int keep) {
+      if (issued - signaled <= keep) return;
+      cp_async_wait_upto(keep);
+      fence_proxy_async_smem();
+      for (; signaled < issued - keep; ++signaled) mbar_arrive(&kv_full[signaled % kStages]);
+    };
+    load_idx(0);
+    for (int j = 0; j < nchunks; ++j) {
+      const int st = j % kStages;
       int iv[kN / 4];
 #pragma unroll
       for (int m = 0; m < kN / 4; ++m) iv[m] = ivn[m];
-      if (!mbar_wait(&kv_empty[w], (use & 1) ^ 1, p.wait_ns, ab)) { fail(1); break; }
+      if (j >= kStages) {
+        const uint32_t par = ((j / kStages) - 1) & 1;
+        // publish everything first when the stage is not free yet
+        if (!__all_sync(0xffffffffu, mbar_test_wait(&kv_empty[st], par))) {
+          retire(0);
+          if (!wwait(&kv_empty[st], par)) { fail(1); break; }
+        }
+      }
+      uint8_t* stage = sKV + st * C::STAGE;
+      uint32_t mask = 0;
 #pragma unroll
       for (int m = 0; m < kN / 4; ++m) {
         const int r = rg + 4 * m;
@@ -197,7 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           v = -1;
         }
         const bool valid = v >= 0;
-        if (c16 == 0) sMeta[w * kN + r] = valid ? 1 : 0;
+        // lanes 0, 8, 16, 24 hold rows 4m .. 4m+3
+        const uint32_t bal = __ballot_sync(0xffffffffu, valid);
+        mask |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u)) << (4 * m);
         const uint16_t* src = kvb + (size_t)(valid ? v : 0) * DK;
 #pragma unroll
         for (int a = 0; a < C::NATOM; ++a) {
@@ -205,13 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_async16(stage + a * C::KV_ATOM + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
         }
       }
+      if (lane == 0) sMask[st] = mask;
       cp_async_commit();
-      load_idx(j + kStages);
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(&kv_full[w]);
+      ++issued;
+      load_idx(j + 1);
+      retire(kInFlight - 1);
     }
-    cp_async_wait<0>();
+    retire(0);
     // drain: the Q load must have landed before this CTA's memory is reused
     if (q_issued) mbar_wait(q_full, 0, p.wait_ns, no_abort);
   } else if (warp == kMmaWarp) {
@@ -219,57 +268,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(kFmtBF16, kFmtBF16, 0, 0, 128, kN);
       constexpr uint32_t idesc_pv = make_idesc(kFmtBF16, kFmtBF16, 0, 1, 128, C::DVH);
-      const uint32_t q_base = smem_u32(sQ), kv_base = smem_u32(sKV), p_base = smem_u32(sP);
-      const uint32_t v_atom = (uint32_t)(half * C::DVH / 64);
-      int pv_issued = 0;
-      auto issue_pv = [&](int i) {
-        tc_fence_after();
-        const int st = i & 1;
-        const uint32_t vbase = kv_base + st * C::STAGE + v_atom * C::KV_ATOM;
-        const uint64_t pdesc = make_sdesc(p_base, 16, 512, kSwizzle64);
-#pragma unroll
-        for (int ks = 0; ks < kN / 16; ++ks) {
-          const uint64_t vdesc = make_sdesc(vbase + ks * 16 * 128, C::KV_ATOM, 1024, kSwizzle128);
-          mma_bf16(tmem + kOCol, pdesc + 2 * ks, vdesc, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(pv_done);
-        mma_commit(&kv_empty[st]);
-        pv_issued = i + 1;
-      };
-      bool ok = nchunks == 0 || mbar_wait(q_full, 0, p.wait_ns, ab);
+      // descriptors are built once; a step only adds its byte offset >> 4 to
+      // the start-address field (no carry: shared addresses are < 256 KB)
+      const uint64_t kdesc0 = make_sdesc(smem_u32(sKV), 16, 1024, kSwizzle128);
+      const uint64_t qdesc0 = make_sdesc(smem_u32(sQ), 16, 1024, kSwizzle128);
+      const uint64_t vdesc0 =
+          make_sdesc(smem_u32(sKV) + (uint32_t)(half * C::DVH / 64) * C::KV_ATOM, C::KV_ATOM, 1024, kSwizzle128);
+      bool ok = nchunks == 0 || ((C::QS_ATOMS == 0 || mbar_wait(q_full, 0, p.wait_ns, ab)) &&
+                                 mbar_wait(q_ready, 0, p.wait_ns, ab));
       if (!ok) fail(3);
       // Issue whichever MMA is ready: Q K^T of chunk qk once its rows have
-      // landed (and its S buffer is free), P V of chunk pv once its
-      // probabilities are written.  P V never waits behind a later chunk's
-      // gather, so a stage is handed back to its gather warp as early as the
-      // data dependencies allow.
+      // landed and P V of chunk qk - kSBuf has freed its S buffer; P V of
+      // chunk pv once its probabilities are written.
       int qk = 0, pv = 0;
       uint64_t t_idle = 0;
       uint32_t spins = 0;
       while (ok && pv < nchunks) {
         bool progressed = false;
-        if (qk < nchunks && qk <= pv + 1) {
-          const int st = qk & 1;
-          if (mbar_test_wait(&kv_full[st], (qk >> 1) & 1) &&
-              (qk < 2 || mbar_test_wait(&s_free[st], ((qk >> 1) - 1) & 1))) {
+        if (qk < nchunks && qk < pv + kSBuf) {
+          const int st = qk % kStages, sb = qk % kSBuf;
+          if (mbar_test_wait(&kv_full[st], (qk / kStages) & 1) &&
+              (qk < kSBuf || mbar_test_wait(&pv_done[sb], ((qk / kSBuf) - 1) & 1))) {
             fence_proxy_async_smem();
             tc_fence_after();
-            const uint32_t sbase = kv_base + st * C::STAGE;
-#pragma unroll 4
+            const uint64_t kst = kdesc0 + (uint64_t)((st * C::STAGE) >> 4);
+            const uint32_t dS = tmem + C::SCOL + sb * kN;
+#pragma unroll
             for (int ks = 0; ks < C::KSTEPS; ++ks) {
               const int d = ks * 16;
-              const uint32_t off = (uint32_t)((d % 64) * 2);
-              const uint64_t adesc = make_sdesc(q_base + (d / 64) * C::Q_ATOM + off, 16, 1024, kSwizzle128);
-              const uint64_t bdesc = make_sdesc(sbase + (d / 64) * C::KV_ATOM + off, 16, 1024, kSwizzle128);
-              mma_bf16(tmem + kSCol + st * kN, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+              const uint64_t bdesc = kst + (uint64_t)(((d / 64) * C::KV_ATOM + (d % 64) * 2) >> 4);
+              if (ks < C::QT_STEPS) {
+                mma_bf16_ts(dS, tmem + C::QCOL + ks * 8, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+              } else {
+                const int dq = d - C::QT_DIMS;
+                const uint64_t adesc = qdesc0 + (uint64_t)(((dq / 64) * C::Q_ATOM + (dq % 64) * 2) >> 4);
+                mma_bf16(dS, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+              }
             }
-            mma_commit(&s_full[st]);
+            mma_commit(&s_full[sb]);
             ++qk;
             progressed = true;
           }
         }
-        if (pv < qk && mbar_test_wait(p_full, pv & 1)) {
-          issue_pv(pv);
+        if (pv < qk && mbar_test_wait(&p_full[pv % kSBuf], (pv / kSBuf) & 1)) {
+          tc_fence_after();
+          const int st = pv % kStages, sb = pv % kSBuf;
+          const uint64_t vst = vdesc0 + (uint64_t)((st * C::STAGE) >> 4);
+#pragma unroll
+          for (int ks = 0; ks < kN / 16; ++ks) {
+            // A = P rows (TMEM, 8 columns = 16 BF16 keys per step), B = V (MN-major)
+            const uint64_t vdesc = vst + (uint64_t)((ks * 16 * 128) >> 4);
+            mma_bf16_ts(tmem + C::OCOL, tmem + C::SCOL + sb * kN + ks * 8, vdesc, idesc_pv,
+                        (pv > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(&pv_done[sb]);
+          mma_commit(&kv_empty[st]);
           ++pv;
           progressed = true;
         }
@@ -280,9 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // nothing ready: doze briefly on the event most likely next, with
         // bounded idle time, and abort when another role failed
         if (pv < qk)
-          mbar_try_wait_hint(p_full, pv & 1, 200);
+          mbar_try_wait_hint(&p_full[pv % kSBuf], (pv / kSBuf) & 1, 200);
         else
-          mbar_try_wait_hint(&kv_full[qk & 1], (qk >> 1) & 1, 200);
+          mbar_try_wait_hint(&kv_full[qk % kStages], (qk / kStages) & 1, 200);
         if (++spins == 1) t_idle = global_ns();
         if ((spins & 1023u) == 0u) {
           if (*abort_flag != 0) { ok = false; break; }
@@ -295,51 +348,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
-      // drain: the last releases of each stage are never waited by the gather
-      // warps; make sure they have landed before this CTA's memory is reused
-      for (int i = max(0, pv_issued - kStages); i < pv_issued; ++i)
-        mbar_wait(&kv_empty[i & 1], (i >> 1) & 1, p.wait_ns, no_abort);
+      // drain: the last arrivals of each commit barrier are not always waited
+      // by their consumers; make sure they have landed before the CTA exits
+      for (int i = max(0, pv - kStages); i < pv; ++i)
+        mbar_wait(&kv_empty[i % kStages], (i / kStages) & 1, p.wait_ns, no_abort);
+      for (int i = max(0, pv - kSBuf); i < pv; ++i)
+        mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
+      for (int i = max(0, qk - kSBuf); i < qk; ++i)
+        mbar_wait(&s_full[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;              // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    // every lane polls; the warp proceeds only if all lanes saw the phase
-    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-      const bool r = mbar_wait(bar, parity, p.wait_ns, ab);
-      return __all_sync(0xffffffffu, r);
-    };
+    const bool head_ok = row_ok && h < p.H;
+    // Q dims [0, QT_DIMS) of row h into TMEM as BF16 pairs (zeros past H)
+    {
+      const uint16_t* qrow = p.q + ((size_t)(head_ok ? row : 0) * p.H + (head_ok ? h : 0)) * DK;
+      for (int qb = 0; qb < C::QT_BLOCKS; ++qb) {
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int col = qb * 64 + i * 8;
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (head_ok && col < C::QT_DIMS) x = *reinterpret_cast<const uint4*>(qrow + col);
+          v[4 * i] = x.x;
+          v[4 * i + 1] = x.y;
+          v[4 * i + 2] = x.z;
+          v[4 * i + 3] = x.w;
+        }
+        tmem_st32(tmem + lane_addr + C::QCOL + qb * 32, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    const float sc = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nchunks && ok; ++j) {
-      const int sb = j & 1, st = j & 1;
-      // 1. logits of this chunk
-      if (!wwait(&s_full[sb], (j >> 1) & 1)) { fail(6); ok = false; break; }
+      const int sb = j % kSBuf, st = j % kStages;
+      // 1. logits of this chunk and its valid slots
+      if (!wwait(&s_full[sb], (j / kSBuf) & 1)) { fail(6); ok = false; break; }
+      if (!wwait(&kv_full[st], (j / kStages) & 1)) { fail(7); ok = false; break; }
+      const uint32_t mask = sMask[st];
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(tmem + lane_addr + kSCol + sb * kN, sr);
+      const uint32_t saddr = tmem + lane_addr + C::SCOL + sb * kN;
+      uint32_t sr[kN];
+      tmem_ld32(saddr, sr);
       tmem_wait_ld_dep(sr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      // 2. mask the empty slots, update the running maximum
-      if (!wwait(&kv_full[st], (j >> 1) & 1)) { fail(7); ok = false; break; }
-      const uint4* meta = reinterpret_cast<const uint4*>(sMeta + st * kN);
-      float s[kN];
-      float mc = -INFINITY;
+      // 2. running maximum (log2 units; the scale is positive)
+      float mraw = -INFINITY;
+      if (mask == 0xffffffffu) {
 #pragma unroll
-      for (int c = 0; c < kN / 16; ++c) {
-        const uint4 mv = meta[c];
-        const uint32_t words[4] = {mv.x, mv.y, mv.z, mv.w};
+        for (int q = 0; q < kN; ++q) mraw = fmaxf(mraw, __uint_as_float(sr[q]));
+      } else {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const bool valid = (words[q >> 2] >> ((q & 3) * 8)) & 0xffu;
-          const float x = valid ? __uint_as_float(sr[c * 16 + q]) * p.scale_log2 : -INFINITY;
-          s[c * 16 + q] = x;
-          mc = fmaxf(mc, x);
-        }
+        for (int q = 0; q < kN; ++q)
+          if ((mask >> q) & 1u) mraw = fmaxf(mraw, __uint_as_float(sr[q]));
       }
+      const float mc = mraw * sc;
       float alpha = 1.f;
       bool rescale = false;
       if (m_used == -INFINITY) {
@@ -349,50 +419,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_used = mc;
         rescale = true;
       }
-      // 3. the previous P.V is done: P buffer free, accumulator stable
-      if (j >= 1 && !wwait(pv_done, (j - 1) & 1)) { fail(8); ok = false; break; }
-      // 4. rescale the output accumulator when the maximum moved (warp-wide)
+      // 3. rescale the output accumulator when the maximum moved (warp-wide),
+      //    once the previous P V has landed in it
       if (__any_sync(0xffffffffu, rescale)) {
+        if (j >= 1 && !wwait(&pv_done[(j - 1) % kSBuf], ((j - 1) / kSBuf) & 1)) { fail(8); ok = false; break; }
         tc_fence_after();
         for (int c = 0; c < C::DVH / 32; ++c) {
           uint32_t o[32];
-          __syncwarp();
-          tmem_ld32(tmem + lane_addr + kOCol + c * 32, o);
+          tmem_ld32(tmem + lane_addr + C::OCOL + c * 32, o);
           tmem_wait_ld_dep(o);
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(tmem + lane_addr + kOCol + c * 32, o);
+          tmem_st32(tmem + lane_addr + C::OCOL + c * 32, o);
         }
         tmem_wait_st();
       }
-      // 5. probabilities (bf16) into P with the 64-byte swizzle: 16-byte
-      //    chunk c of row h lands at h*64 + ((c ^ ((h >> 1) & 3)) * 16)
+      // 4. probabilities as BF16 pairs over the first kN/2 columns of the S
+      //    buffer (already read above)
       float rs = 0.f;
-      uint8_t* prow = sP + h * 64;
-      const bool any = m_used != -INFINITY;
+      uint32_t pk[kN / 2];
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float e[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          e[q] = any ? exp2f(s[c * 8 + q] - m_used) : 0.f;
-          rs += e[q];
-        }
-        uint4 pk;
-        pk.x = pack_bf16x2(e[0], e[1]);
-        pk.y = pack_bf16x2(e[2], e[3]);
-        pk.z = pack_bf16x2(e[4], e[5]);
-        pk.w = pack_bf16x2(e[6], e[7]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ ((h >> 1) & 3)) << 4)) = pk;
+      for (int q = 0; q < kN / 2; ++q) {
+        float e0 = exp2f(fmaf(__uint_as_float(sr[2 * q]), sc, neg_m));
+        float e1 = exp2f(fmaf(__uint_as_float(sr[2 * q + 1]), sc, neg_m));
+        if (!((mask >> (2 * q)) & 1u) || m_used == -INFINITY) e0 = 0.f;
+        if (!((mask >> (2 * q + 1)) & 1u) || m_used == -INFINITY) e1 = 0.f;
+        rs += e0 + e1;
+        pk[q] = pack_bf16x2(e0, e1);
       }
+      tmem_st16(saddr, pk);
+      tmem_wait_st();
       l = l * alpha + rs;
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    // 6. output
-    if (ok && nchunks > 0 && !wwait(pv_done, (nchunks - 1) & 1)) {
+    // 5. output
+    if (ok && nchunks > 0 && !wwait(&pv_done[(nchunks - 1) % kSBuf], ((nchunks - 1) / kSBuf) & 1)) {
       fail(9);
       ok = false;
     }
@@ -400,14 +464,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m_used + log2f(l) : -INFINITY;
-      const bool write_o = h < p.H;
       const int vlo = half * C::DVH;
       for (int c = 0; c < C::DVH / 32; ++c) {
         uint32_t o[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_addr + kOCol + c * 32, o);
+        tmem_ld32(tmem + lane_addr + C::OCOL + c * 32, o);
         tmem_wait_ld_dep(o);
-        if (!write_o) continue;
+        if (!head_ok) continue;
         if (p.nsplit == 1) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)row * p.H + h) * DV + vlo + c * 32);
 #pragma unroll
@@ -428,14 +490,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __uint_as_float(o[4 * g + 2]) * inv, __uint_as_float(o[4 * g + 3]) * inv);
         }
       }
-      if (half == 0 && h < p.H) {
+      if (half == 0 && head_ok) {
         if (p.nsplit == 1) {
           if (p.lse != nullptr) p.lse[(size_t)row * p.H + h] = lse2 * 0.6931471805599453f;
         } else {
           p.part_lse[((size_t)row * p.nsplit + split) * p.H + h] = lse2;
         }
       }
-    } else if (ok && h < p.H && row_ok && half == 0) {
+    } else if (ok && head_ok && half == 0) {
       // no selected slots in this split: empty result
       if (p.nsplit > 1) p.part_lse[((size_t)row * p.nsplit + split) * p.H + h] = -INFINITY;
     }
@@ -490,6 +552,7 @@ template <int DK, int DV>
 cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   using Cf = Cfg<DK, DV>;
   AttnParams p;
+  p.q = a.q;
   p.kv = a.kv;
   p.idx = a.idx;
   p.out = a.out;
@@ -508,6 +571,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   p.part_o = a.part;
   p.part_lse = a.part ? a.part + (size_t)rows * a.nsplit * a.H * DV : nullptr;
   // Q as a [rows * H, DK] BF16 matrix read in 128-row x 64-column boxes
+  // (only the atoms kept in shared memory are loaded this way)
   CUtensorMap tm_q;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, (uint64_t)rows * a.H, DK, (uint64_t)DK * 2, 128,
                     64, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -532,10 +596,13 @@ size_t attn_partial_floats(int rows, int H, int d_v, int nsplit) {
   return nsplit > 1 ? (size_t)rows * nsplit * H * (d_v + 1) : 0;
 }
 
-int attn_choose_nsplit(int rows, int H, int k, int num_sms) {
+int attn_choose_nsplit(int rows, int H, int d_v, int k, int num_sms) {
   (void)H;
+  // one wave: rows x CTAs per query (value halves) x splits <= SM count
+  // (one CTA per SM), at least one split, at most one chunk per split
+  const int per_row = rows * (d_v >= 128 ? 2 : 1);
   const int chunks = (k + kN - 1) / kN;
-  int target = rows > 0 ? (num_sms + rows - 1) / rows : 1;
+  int target = per_row > 0 ? num_sms / per_row : 1;
   if (target < 1) target = 1;
   if (target > chunks) target = chunks;
   const int kc = ((k + target - 1) / target + kN - 1) / kN * kN;

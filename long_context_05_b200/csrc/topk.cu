@@ -172,8 +172,8 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
   __syncthreads();
   const bool fits = keys_in_bin <= (unsigned int)kCap;
   // pass 2: keys above bin B go straight out; bin B keys become candidates
-  for (int x = tid; x < n; x += kThreads) {
-    const unsigned int key = order_key(row[x]);
+  auto visit = [&](float f, int x) {
+    const unsigned int key = order_key(f);
     const unsigned int bin = key >> kBinShift;
     if (bin > B) {
       put(out, k, atomicAdd(&sm.cnt, 1), x, err, 1);
@@ -186,6 +186,34 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
         report_error(err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_TOPK | (7u << 8));
       }
     }
+  };
+  {
+    // 16-byte loads over the aligned body (rows start 16-byte aligned), two
+    // in flight per thread; scalar tail
+    const int n4 = n / 4;
+    const float4* r4 = reinterpret_cast<const float4*>(row);
+    int x = tid;
+    for (; x + kThreads < n4; x += 2 * kThreads) {
+      float4 v[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) v[u] = r4[x + u * kThreads];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int e = 4 * (x + u * kThreads);
+        visit(v[u].x, e);
+        visit(v[u].y, e + 1);
+        visit(v[u].z, e + 2);
+        visit(v[u].w, e + 3);
+      }
+    }
+    for (; x < n4; x += kThreads) {
+      const float4 v = r4[x];
+      visit(v.x, 4 * x);
+      visit(v.y, 4 * x + 1);
+      visit(v.z, 4 * x + 2);
+      visit(v.w, 4 * x + 3);
+    }
+    for (int e = 4 * n4 + tid; e < n; e += kThreads) visit(row[e], e);
   }
   __syncthreads();
   unsigned int thr, krem;
@@ -275,7 +303,22 @@ __device__ void histogram_pass(const float* row, int lo, int hi, unsigned int* h
   }
   for (int x = lo + (int)threadIdx.x; x < a0; x += kThreads) atomicAdd(&hist[order_key(row[x]) >> kBinShift], 1u);
   const float4* r4 = reinterpret_cast<const float4*>(row + a0);
-  for (int x = threadIdx.x; x < (a1 - a0) / 4; x += kThreads) {
+  const int n4 = (a1 - a0) / 4;
+  int x = threadIdx.x;
+  // four independent 16-byte loads in flight per thread
+  for (; x + 3 * kThreads < n4; x += 4 * kThreads) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = r4[x + u * kThreads];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      atomicAdd(&hist[order_key(v[u].x) >> kBinShift], 1u);
+      atomicAdd(&hist[order_key(v[u].y) >> kBinShift], 1u);
+      atomicAdd(&hist[order_key(v[u].z) >> kBinShift], 1u);
+      atomicAdd(&hist[order_key(v[u].w) >> kBinShift], 1u);
+    }
+  }
+  for (; x < n4; x += kThreads) {
     const float4 v = r4[x];
     atomicAdd(&hist[order_key(v.x) >> kBinShift], 1u);
     atomicAdd(&hist[order_key(v.y) >> kBinShift], 1u);
@@ -286,7 +329,7 @@ __device__ void histogram_pass(const float* row, int lo, int hi, unsigned int* h
 }
 
 // One block per row.
-__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(TopkArgs a, DevErr* err) {
+__global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   int b, t, n;
@@ -333,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, 
     if (hist[x]) atomicAdd(&gh[x], hist[x]);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_seg_select_kernel(TopkArgs a, unsigned int* ghist, DevErr* err) {
+__global__ void __launch_bounds__(kThreads, 2) topk_seg_select_kernel(TopkArgs a, unsigned int* ghist, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   int b, t, n;

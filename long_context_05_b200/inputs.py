@@ -96,6 +96,11 @@ WORKLOADS = {
     "prefill_128k": Workload("prefill_128k", B=1, T=131072, S=131072, H_I=64, D_I=128,
                              H=128, d_k=576, d_v=512, k=2048, q_block=4096, seed=1004,
                              needles=64, local_window=512),
+    # the last 512 queries of a 128K prefill (a chunked-prefill step): full
+    # 128K score rows at a size small enough for a profiler capture
+    "prefill_chunk_128k": Workload("prefill_chunk_128k", B=1, T=512, S=131072, H_I=64, D_I=128,
+                                   H=128, d_k=576, d_v=512, k=2048, q_block=512, seed=1005,
+                                   needles=64, local_window=512),
 }
 
 # rows generated per random draw; fixed so the stream does not depend on memory
