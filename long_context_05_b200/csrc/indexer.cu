@@ -40,6 +40,7 @@ constexpr int kMaxNB = 8;      // sub-tiles per work item
 constexpr int kKC = 32;        // key tiles per work item (at most; fewer when items are scarce)
 constexpr int kStages = 4;     // depth of the k_I ring
 constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * kNSub = 512 columns)
+static_assert((kNAcc & (kNAcc - 1)) == 0, "accumulator index is taken with a mask");
 constexpr int kEpiGroups = 3;   // epilogue groups of four warps
 constexpr int kEpiThreads = 128 * kEpiGroups;
 constexpr int kThreads = 64 + kEpiThreads;
@@ -108,14 +109,23 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
   }
 }
 
-// sub-tile j of an item covers queries [t0 + j*QPS, min(t0 + (j+1)*QPS, tend))
+// Sub-tile j of an item covers queries [t0 + j*QPS, min(t0 + (j+1)*QPS, tend)).
+// nsub: sub-tiles holding at least one query of the item.  For key tile kt
+// the active sub-tiles (some query sees a key of the tile) are [jlo, nsub):
+// the last query of sub-tile j grows with j, and the item's last query sees
+// every key tile the item covers.
 template <int HI>
-__device__ __forceinline__ bool subtile_active(const IdxParams& p, const Item& it, int j, int kt) {
+__device__ __forceinline__ int item_nsub(const IdxParams& p, const Item& it) {
   constexpr int QPS = kNSub / HI;
-  const int qa = it.t0 + j * QPS;
-  if (qa >= it.tend) return false;
-  const int qlast = min(qa + QPS, it.tend) - 1;
-  return kt * kBM <= p.S - p.T + qlast;
+  return min(p.nb, (it.tend - it.t0 + QPS - 1) / QPS);
+}
+template <int HI>
+__device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, int kt, int nsub) {
+  constexpr int QPS = kNSub / HI;
+  // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM - (S - T)
+  const int x = kt * kBM - (p.S - p.T) - it.t0 + QPS;
+  const int j = x > 0 ? x / QPS - 1 : 0;
+  return j < 0 ? 0 : (j < nsub - 1 ? j : nsub - 1);
 }
 
 template <int DI, int HI>
@@ -219,25 +229,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc(kFmtE4M3, kFmtE4M3, 0, 0, kBM, kNSub);
       uint32_t a_cnt = 0, items = 0, u = 0;
-      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      // descriptors built once; a stage or sub-tile only adds its offset >> 4
+      const uint64_t adesc0 = make_sdesc(smem_u32(sA), 16, L::kSBO, L::kSwizzleLayout);
+      const uint64_t bdesc0 = make_sdesc(smem_u32(sB), 16, L::kSBO, L::kSwizzleLayout);
       for_each_item<HI>(p, [&](const Item& it) {
         if (!mbar_wait(b_full, items & 1, p.wait_ns, ab)) { fail(3); return false; }
         ++items;
+        const int nsub = item_nsub<HI>(p, it);
         const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
           const int st = a_cnt % kStages;
           if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.wait_ns, ab)) { fail(4); return false; }
           tc_fence_after();
-          const uint64_t adesc = make_sdesc(a_base + st * L::kABytes, 16, L::kSBO, L::kSwizzleLayout);
-          for (int j = 0; j < p.nb; ++j) {
-            if (!subtile_active<HI>(p, it, j, kt)) continue;
-            const int acc = u % kNAcc;
-            if (!mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.wait_ns, ab)) { fail(5); return false; }
+          const uint64_t adesc = adesc0 + (uint64_t)((st * L::kABytes) >> 4);
+          for (int j = first_active<HI>(p, it, kt, nsub); j < nsub; ++j) {
+            const int acc = u & (kNAcc - 1);
+            if (!mbar_test_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1) &&
+                !mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.wait_ns, ab)) {
+              fail(5);
+              return false;
+            }
             tc_fence_after();
-            const uint64_t bdesc = make_sdesc(b_base + j * L::kBSubBytes, 16, L::kSBO, L::kSwizzleLayout);
+            const uint64_t bdesc = bdesc0 + (uint64_t)((j * L::kBSubBytes) >> 4);
+            const uint32_t dacc = tmem_base + acc * kNSub;
 #pragma unroll
             for (int ks = 0; ks < DI / 32; ++ks)
-              mma_f8(tmem_base + acc * kNSub, adesc + 2 * ks, bdesc + 2 * ks, idesc, ks > 0 ? 1u : 0u);
+              mma_f8(dacc, adesc + 2 * ks, bdesc + 2 * ks, idesc, ks > 0 ? 1u : 0u);
             mma_commit(&acc_full[acc]);
             ++u;
           }
@@ -272,15 +289,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&w_ready[items & 1]);
       if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.wait_ns, ab)) { fail(7); return false; }
       ++items;
+      const int nsub = item_nsub<HI>(p, it);
       const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
       for (int kt = kt0; kt < kt1; ++kt) {
         const int s = kt * kBM + r;
         const float ks = s < p.S ? p.k_scale[(size_t)it.b * p.S + s] : 0.f;
-        for (int j = 0; j < p.nb; ++j) {
-          if (!subtile_active<HI>(p, it, j, kt)) continue;
-          const uint32_t my = u++;
-          if ((int)(my % kEpiGroups) != grp) continue;
-          const int acc = my % kNAcc;
+        const int jlo = first_active<HI>(p, it, kt, nsub);
+        const uint32_t u0 = u;
+        u += (uint32_t)(nsub - jlo);
+        // this group's sub-tiles of the tile: my = u0 + (j - jlo) == grp (mod kEpiGroups)
+        const int skip = (int)((grp + kEpiGroups - (int)(u0 % kEpiGroups)) % kEpiGroups);
+        for (int j = jlo + skip; j < nsub; j += kEpiGroups) {
+          const uint32_t my = u0 + (uint32_t)(j - jlo);
+          const int acc = my & (kNAcc - 1);
           const bool got = mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.wait_ns, ab);
           if (!__all_sync(0xffffffffu, got)) { fail(6); return false; }
           tc_fence_after();
