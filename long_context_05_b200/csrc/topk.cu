@@ -157,6 +157,49 @@ __device__ __forceinline__ void put(int32_t* out, int k, int pos, int value, Dev
   }
 }
 
+// Exact selection among nc candidate keys held in shared memory (sm.ck,
+// sm.ci), all sharing the bits `mask` with `prefix` (bits below `hi` free):
+// emit the `need` largest, ties to the lower index, after the sm.cnt slots
+// already written.
+__device__ void select_candidates(int nc, unsigned int prefix, unsigned int mask, int hi, unsigned int need, int k,
+                                  int32_t* out, Smem& sm, DevErr* err) {
+  const int tid = threadIdx.x;
+  const unsigned int* ck = sm.ck;
+  unsigned int krem;
+  const unsigned int thr = radix_select([ck](int i) { return ck[i]; }, nc, prefix, mask, hi, need, sm.hist,
+                                        sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
+  // candidates above thr
+  unsigned int eq_local = 0;
+  for (int i = tid; i < nc; i += kThreads) {
+    if (sm.ck[i] > thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 2);
+    eq_local += sm.ck[i] == thr;
+  }
+  block_scan(eq_local, sm.warp_tot, &sm.total);
+  const unsigned int E = sm.total;
+  if (E == krem) {
+    for (int i = tid; i < nc; i += kThreads)
+      if (sm.ck[i] == thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 3);
+    return;
+  }
+  // more equal keys than slots: keep the lowest indices.  Gather the equal
+  // candidates' indices and select on ~index (lower index = larger key).
+  if (tid == 0) sm.eq_base = 0;
+  __syncthreads();
+  for (int i = tid; i < nc; i += kThreads)
+    if (sm.ck[i] == thr) {
+      const int p = atomicAdd(&sm.eq_base, 1);
+      if (p < kCap) sm.eqi[p] = sm.ci[i];
+    }
+  __syncthreads();
+  const int ne = min(sm.eq_base, kCap);
+  const int* ci = sm.eqi;
+  unsigned int krem2;
+  const unsigned int ithr = radix_select([ci](int i) { return ~(unsigned int)ci[i]; }, ne, 0u, 0u, 32, krem, sm.hist,
+                                         sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem2);
+  for (int i = tid; i < ne; i += kThreads)
+    if (~(unsigned int)sm.eqi[i] >= ithr) put(out, k, atomicAdd(&sm.cnt, 1), sm.eqi[i], err, 4);
+}
+
 __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, unsigned int B, unsigned int above,
                                 unsigned int keys_in_bin, Smem& sm, DevErr* err) {
   const int tid = threadIdx.x;
@@ -218,40 +261,7 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
   __syncthreads();
   unsigned int thr, krem;
   if (fits) {
-    const int nc = min(sm.ncand, kCap);
-    const unsigned int* ck = sm.ck;
-    thr = radix_select([ck](int i) { return ck[i]; }, nc, B << kBinShift, 0xFFFFFFFFu << kBinShift, kBinShift,
-                       need, sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
-    // candidates above thr
-    unsigned int eq_local = 0;
-    for (int i = tid; i < nc; i += kThreads) {
-      if (sm.ck[i] > thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 2);
-      eq_local += sm.ck[i] == thr;
-    }
-    block_scan(eq_local, sm.warp_tot, &sm.total);
-    const unsigned int E = sm.total;
-    if (E == krem) {
-      for (int i = tid; i < nc; i += kThreads)
-        if (sm.ck[i] == thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 3);
-      return;
-    }
-    // more equal keys than slots: keep the lowest indices.  Gather the equal
-    // candidates' indices and select on ~index (lower index = larger key).
-    if (tid == 0) sm.eq_base = 0;
-    __syncthreads();
-    for (int i = tid; i < nc; i += kThreads)
-      if (sm.ck[i] == thr) {
-        const int p = atomicAdd(&sm.eq_base, 1);
-        if (p < kCap) sm.eqi[p] = sm.ci[i];
-      }
-    __syncthreads();
-    const int ne = min(sm.eq_base, kCap);
-    const int* ci = sm.eqi;
-    unsigned int krem2;
-    const unsigned int ithr = radix_select([ci](int i) { return ~(unsigned int)ci[i]; }, ne, 0u, 0u, 32, krem,
-                                           sm.hist, sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem2);
-    for (int i = tid; i < ne; i += kThreads)
-      if (~(unsigned int)sm.eqi[i] >= ithr) put(out, k, atomicAdd(&sm.cnt, 1), sm.eqi[i], err, 4);
+    select_candidates(min(sm.ncand, kCap), B << kBinShift, 0xFFFFFFFFu << kBinShift, kBinShift, need, k, out, sm, err);
     return;
   }
   // bin B too large for shared memory: radix passes over the row itself
@@ -328,6 +338,83 @@ __device__ void histogram_pass(const float* row, int lo, int hi, unsigned int* h
   for (int x = a1 + (int)threadIdx.x; x < hi; x += kThreads) atomicAdd(&hist[order_key(row[x]) >> kBinShift], 1u);
 }
 
+// One pass over the row when a lower bound on the k-th key is known: every
+// key at or above `lo` becomes a candidate.  Rows of at most kCap keys take
+// all keys; longer rows estimate the bound from a sample (four adjacent keys
+// out of every 64 x step, about 1.5 k / (16 step) + 16 sampled keys above
+// it, so about 1.5 k keys of the row are expected above it).  Returns false
+// (nothing written) when the candidates are fewer than k or do not fit in
+// shared memory; the caller then runs the two-pass histogram path.
+__device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& sm, DevErr* err) {
+  const int tid = threadIdx.x;
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  unsigned int lo = 0u;
+  if (n > kCap) {
+    const int nblk = n / 64;                         // 64-key blocks (>= 128 here)
+    const int step = (nblk + kCap / 4 - 1) / (kCap / 4);
+    const int ns = nblk / step;                      // sampled blocks, <= kCap / 4
+    const int m = 4 * ns;
+    const int rs = min(m, (3 * k) / (2 * 16 * step) + 16);
+    for (int i = tid; i < ns; i += kThreads) {
+      const float4 v = r4[(size_t)i * step * 16];
+      sm.ck[4 * i] = order_key(v.x);
+      sm.ck[4 * i + 1] = order_key(v.y);
+      sm.ck[4 * i + 2] = order_key(v.z);
+      sm.ck[4 * i + 3] = order_key(v.w);
+    }
+    __syncthreads();
+    const unsigned int* ck = sm.ck;
+    unsigned int krem;
+    lo = radix_select([ck](int i) { return ck[i]; }, m, 0u, 0u, 32, (unsigned int)rs, sm.hist, sm.warp_tot, &sm.bin,
+                      &sm.above, &sm.total, &krem);
+  }
+  if (tid == 0) {
+    sm.cnt = 0;
+    sm.ncand = 0;
+  }
+  __syncthreads();
+  auto visit = [&](float f, int x) {
+    const unsigned int key = order_key(f);
+    if (key >= lo) {
+      const int p = atomicAdd(&sm.ncand, 1);
+      if (p < kCap) {
+        sm.ck[p] = key;
+        sm.ci[p] = x;
+      }
+    }
+  };
+  {
+    const int n4 = n / 4;
+    int x = tid;
+    for (; x + kThreads < n4; x += 2 * kThreads) {
+      float4 v[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) v[u] = r4[x + u * kThreads];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int e = 4 * (x + u * kThreads);
+        visit(v[u].x, e);
+        visit(v[u].y, e + 1);
+        visit(v[u].z, e + 2);
+        visit(v[u].w, e + 3);
+      }
+    }
+    for (; x < n4; x += kThreads) {
+      const float4 v = r4[x];
+      visit(v.x, 4 * x);
+      visit(v.y, 4 * x + 1);
+      visit(v.z, 4 * x + 2);
+      visit(v.w, 4 * x + 3);
+    }
+    for (int e = 4 * n4 + tid; e < n; e += kThreads) visit(row[e], e);
+  }
+  __syncthreads();
+  const int nc = sm.ncand;
+  if (nc < k || nc > kCap) return false;
+  select_candidates(nc, 0u, 0u, 32, (unsigned int)k, k, out, sm, err);
+  return true;
+}
+
 // One block per row.
 __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -341,6 +428,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevEr
     for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
     return;
   }
+  if (single_pass(row, n, k, out, sm, err)) return;
+  // two passes: histogram of the top 11 bits, then the threshold bin
+  __syncthreads();
   for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = 0u;
   if (threadIdx.x == 0) sm.bin = 0xFFFFFFFFu;
   __syncthreads();
