@@ -14,28 +14,34 @@
 // (Q K^T over the 576-wide key) and its 128 x 256 half of the output.
 //
 // Per CTA:
-//   * TMEM: O (128 x 256 FP32) | two 32-column S buffers | the first 384
-//     columns of Q as BF16 pairs (192 columns) = 512 columns.  The rest of Q
-//     (192 columns, 48 KB) sits in shared memory, loaded once by TMA.  Q K^T
-//     takes its A operand from TMEM for 24 of its 36 K steps, which keeps
-//     those steps off the shared-memory port;
-//   * the rest of shared memory is a 4-stage ring of gathered key rows (32
-//     keys x 1152 B per stage), filled with 16-byte cp.async by one gather
-//     warp that keeps three chunks in flight;
-//   * the softmax writes the BF16 probabilities over the first half of the
-//     chunk's S buffer, and O += P V takes P from TMEM and V as the MN-major
+//   * TMEM: O (128 x 256 FP32) | two 64-column S buffers | the first 256
+//     key dims of Q as BF16 pairs (128 columns) = 512 columns.  The other
+//     320 dims of Q (80 KB) sit in shared memory, loaded once by TMA.  Q K^T
+//     takes its A operand from TMEM for 16 of its 36 K steps;
+//   * the rest of shared memory is a ring of four 32-key slots (1152 B per
+//     key, 128B-swizzled K-major atoms laid out [atom][slot][row] so that the
+//     two slots of a chunk form one 64-row tile).  Each MMA chunk is 64 keys
+//     (N = 64): a tcgen05.mma costs the issuing thread about as much for
+//     N = 32 as for N = 64, so larger N halves the issue time per key;
+//   * six gather warps fill the ring with 16-byte cp.async, three per slot
+//     of a chunk (one issuing warp moves only about 18 B/clk);
+//   * eight softmax warps, two per TMEM lane quarter: each takes 32 of the
+//     chunk's 64 logits, the two exchange their partial row maxima through
+//     shared memory, and each writes its BF16 probabilities over part of the
+//     chunk's S buffer; O += P V takes P from TMEM and V as the MN-major
 //     view of the gathered rows.  With two S/P buffers the softmax of chunk
 //     j+1 runs while P V of chunk j executes.
 // Online softmax in base 2 with a lazy rescale: the running maximum moves
 // only when a chunk exceeds it by more than 8 (so p <= 256), and then the
-// TMEM accumulator is rescaled once, after the previous P V has landed.
+// TMEM accumulator is rescaled once (each softmax warp its half of the value
+// columns), after the previous P V has landed.
 //
-// Warp roles (192 threads): warp 0 gathers, warp 1 owns TMEM and issues the
-// MMAs (whichever is ready: Q K^T of the next chunk or P V of the oldest),
-// warps 2-5 run the softmax (thread = head row) and write the output.
-// Decode splits the selected keys of each query over several CTAs and merges
-// the partial results with a combine kernel.  Every barrier that receives an
-// asynchronous arrival is waited on before the CTA exits.
+// Warp roles (480 threads): warp 0 owns TMEM and issues the MMAs (whichever
+// is ready: Q K^T of the next chunk or P V of the oldest), warps 1-3 and
+// 12-14 gather, warps 4-11 run the softmax (thread = head row) and write the
+// output.  Decode splits the selected keys of each query over several CTAs
+// and merges the partial results with a combine kernel.  Every barrier that
+// receives an asynchronous arrival is waited on before the CTA exits.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -47,12 +53,19 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kN = 32;          // selected keys per chunk (N of Q K^T)
-constexpr int kStages = 4;      // gather ring
-constexpr int kInFlight = 3;    // chunks the gather warp keeps in flight
+constexpr int kSlotKeys = 32;   // keys per gather slot
+constexpr int kSlots = 4;       // gather ring slots
+constexpr int kN = 2 * kSlotKeys;  // keys per chunk = N of Q K^T (two adjacent slots)
 constexpr int kSBuf = 2;        // S/P buffers in TMEM
-constexpr int kThreads = 192;
-constexpr int kGatherWarp = 0, kMmaWarp = 1;
+// Warps: 0 MMA, 1-3 gather the even slot of every chunk, 4-11 softmax (two
+// per TMEM lane quarter: warps 4-7 take keys 0-31 of a chunk, 8-11 keys
+// 32-63), 12-14 gather the odd slot.  One issuing warp moves only about
+// 18 B/clk of 16-byte cp.async; three per slot let both slots of a chunk land
+// in parallel.
+constexpr int kMmaWarp = 0, kFirstSoftmaxWarp = 4, kSoftmaxWarps = 8;
+constexpr int kGatherPerSlot = 3;
+constexpr int kFirstGatherB = kFirstSoftmaxWarp + kSoftmaxWarps;
+constexpr int kThreads = 32 * (kFirstGatherB + kGatherPerSlot);
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -72,16 +85,22 @@ struct Cfg {
   static constexpr int QT_BLOCKS = (QT_DIMS + 63) / 64;  // 32-column stores per row
   static constexpr int QS_ATOMS = (DK - QT_DIMS) / 64;   // Q atoms in shared memory
   static constexpr int Q_ATOM = 128 * 128;               // 128 head rows x 128 bytes
-  static constexpr int KV_ATOM = kN * 128;               // kN key rows x 128 bytes
-  static constexpr int STAGE = NATOM * KV_ATOM;
+  static constexpr int SLOT_ATOM = kSlotKeys * 128;
+  static constexpr int ATOM_STRIDE = kSlots * SLOT_ATOM;
+  static constexpr int RING = NATOM * ATOM_STRIDE;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + QS_ATOMS * Q_ATOM;
-  static constexpr int OFF_MASK = OFF_KV + kStages * STAGE;  // valid-slot bit mask per stage
-  static constexpr int OFF_BAR = OFF_MASK + kStages * 4;
-  static constexpr int NBARS = 2 + 2 * kStages + 3 * kSBuf + 1;
+  static constexpr int OFF_MASK = OFF_KV + RING;
+  // partial row maxima exchanged by the two softmax warps of a lane quarter,
+  // one set per S buffer: [kSBuf][2 sides][128 rows]
+  static constexpr int OFF_XM = OFF_MASK + kSlots * 4;
+  static constexpr int OFF_BAR = OFF_XM + kSBuf * 2 * 128 * 4;
+  static constexpr int NBARS = 2 + 2 * kSlots + 3 * kSBuf + 1 + kSBuf * 4 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int ALLOC = BYTES + 1024;          // room to align the base to 1024
+  // the dynamic shared memory base is checked for 1024-byte alignment at run
+  // time (the swizzled layouts need it), so no slack is allocated
+  static constexpr int ALLOC = BYTES;
   static_assert(DK % 64 == 0 || QT_DIMS == DK, "Q split on whole atoms");
   static_assert(QT_DIMS % 16 == 0 && DVH <= 256 && DVH % 16 == 0, "shape");
   static_assert(QCOL + (QT_DIMS / 2 + 31) / 32 * 32 <= kTmemCols, "TMEM layout");
@@ -104,39 +123,45 @@ struct AttnParams {
   DevErr* err;
 };
 
+// 2^x with the hardware approximation (flushes subnormal results to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// cp.async.wait_group with a run-time count (0 .. kInFlight - 1)
-__device__ __forceinline__ void cp_async_wait_upto(int n) {
-  switch (n) {
-    case 0: cp_async_wait<0>(); break;
-    case 1: cp_async_wait<1>(); break;
-    default: cp_async_wait<2>(); break;
-  }
-}
-static_assert(kInFlight - 1 <= 2, "cp_async_wait_upto range");
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
   using C = Cfg<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (smem_u32(smem_raw) & 1023u) {
+    // self-check: the layouts below need a 1024-byte aligned base
+    if (threadIdx.x == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (0xAu << 8));
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sKV = smem + C::OFF_KV;
   uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;                     // Q atoms in shared memory (TMA)
   uint64_t* q_ready = q_full + 1;              // Q rows in TMEM (4 softmax warps)
-  uint64_t* kv_full = q_ready + 1;             // [kStages] rows landed (32 gather lanes)
-  uint64_t* kv_empty = kv_full + kStages;      // [kStages] stage consumed (MMA commit)
-  uint64_t* s_full = kv_empty + kStages;       // [kSBuf] S written (MMA commit)
+  uint64_t* kv_full = q_ready + 1;
+  uint64_t* kv_empty = kv_full + kSlots;
+  uint64_t* s_full = kv_empty + kSlots;
   uint64_t* p_full = s_full + kSBuf;           // [kSBuf] P written (4 softmax warps)
   uint64_t* pv_done = p_full + kSBuf;          // [kSBuf] P V of the buffer complete (MMA commit)
   uint64_t* mma_done = pv_done + kSBuf;
+  uint64_t* mx_bar = mma_done + 1;             // [kSBuf][4 quarters] both partial maxima written
+  uint64_t* lx_bar = mx_bar + kSBuf * 4;       // [4 quarters] both partial row sums written
+  float* sXM = reinterpret_cast<float*>(smem + C::OFF_XM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -154,17 +179,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_ready, 4);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&kv_full[i], 32);
+    mbar_init(q_ready, kSoftmaxWarps);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&kv_full[i], 32 * kGatherPerSlot);
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], kSoftmaxWarps);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < kSBuf * 4 + 4; ++i) mbar_init(&mx_bar[i], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -189,10 +215,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     return __all_sync(0xffffffffu, r);
   };
 
-  if (warp == kGatherWarp) {
+  if (warp != kMmaWarp && (warp < kFirstSoftmaxWarp || warp >= kFirstGatherB)) {
     // ------------------------------------------------------------ gather
+    // slot half h of every chunk; warp g of the half copies atoms g, g+3, g+6
+    const int h = warp < kFirstSoftmaxWarp ? 0 : 1;
+    const int g = h == 0 ? warp - 1 : warp - kFirstGatherB;
     bool q_issued = false;
-    if (lane == 0 && nchunks > 0 && C::QS_ATOMS > 0) {
+    if (h == 0 && g == 0 && lane == 0 && nchunks > 0 && C::QS_ATOMS > 0) {
       prefetch_tmap(&tm_q);
       mbar_arrive_expect_tx(q_full, C::QS_ATOMS * C::Q_ATOM);
       for (int a = 0; a < C::QS_ATOMS; ++a)
@@ -202,41 +231,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c16 = lane & 7, rg = lane >> 3;  // 16-byte column chunk, row group
     const int32_t* irow = p.idx + (size_t)row * p.k;
     const uint16_t* kvb = p.kv + (size_t)b * p.S * DK;
-    // indices are loaded one chunk ahead, while earlier rows are in flight
-    int ivn[kN / 4];
+    // indices of this half of chunk j, loaded one chunk ahead
+    int ivn[kSlotKeys / 4];
     auto load_idx = [&](int j) {
 #pragma unroll
-      for (int m = 0; m < kN / 4; ++m) {
-        const int slot = slot0 + j * kN + rg + 4 * m;
+      for (int m = 0; m < kSlotKeys / 4; ++m) {
+        const int slot = slot0 + j * kN + h * kSlotKeys + rg + 4 * m;
         ivn[m] = (j < nchunks && slot < slot1) ? irow[slot] : -1;
       }
     };
-    int issued = 0, signaled = 0;
-    // wait until at most `keep` chunks are pending, then publish the others
-    auto retire = [&](int keep) {
-      if (issued - signaled <= keep) return;
-      cp_async_wait_upto(keep);
-      fence_proxy_async_smem();
-      for (; signaled < issued - keep; ++signaled) mbar_arrive(&kv_full[signaled % kStages]);
-    };
     load_idx(0);
     for (int j = 0; j < nchunks; ++j) {
-      const int st = j % kStages;
-      int iv[kN / 4];
+      const int st = 2 * (j % 2) + h;          // ring slot of this half of chunk j
+      int iv[kSlotKeys / 4];
 #pragma unroll
-      for (int m = 0; m < kN / 4; ++m) iv[m] = ivn[m];
-      if (j >= kStages) {
-        const uint32_t par = ((j / kStages) - 1) & 1;
-        // publish everything first when the stage is not free yet
-        if (!__all_sync(0xffffffffu, mbar_test_wait(&kv_empty[st], par))) {
-          retire(0);
-          if (!wwait(&kv_empty[st], par)) { fail(1); break; }
-        }
-      }
-      uint8_t* stage = sKV + st * C::STAGE;
+      for (int m = 0; m < kSlotKeys / 4; ++m) iv[m] = ivn[m];
+      if (j >= 2 && !wwait(&kv_empty[st], (uint32_t)((j / 2) - 1) & 1)) { fail(1); break; }
+      uint8_t* slotp = sKV + st * C::SLOT_ATOM;
       uint32_t mask = 0;
 #pragma unroll
-      for (int m = 0; m < kN / 4; ++m) {
+      for (int m = 0; m < kSlotKeys / 4; ++m) {
         const int r = rg + 4 * m;
         int v = iv[m];
         if (v >= p.S) {
@@ -249,18 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mask |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u)) << (4 * m);
         const uint16_t* src = kvb + (size_t)(valid ? v : 0) * DK;
 #pragma unroll
-        for (int a = 0; a < C::NATOM; ++a) {
-          if (a * 128 + c16 * 16 < DK * 2)
-            cp_async16(stage + a * C::KV_ATOM + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
+        for (int a0 = 0; a0 < C::NATOM; a0 += kGatherPerSlot) {
+          const int a = a0 + g;
+          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2)
+            cp_async16(slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
         }
       }
-      if (lane == 0) sMask[st] = mask;
+      if (g == 0 && lane == 0) sMask[st] = mask;
       cp_async_commit();
-      ++issued;
       load_idx(j + 1);
-      retire(kInFlight - 1);
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(&kv_full[st]);
     }
-    retire(0);
+    cp_async_wait<0>();
     // drain: the Q load must have landed before this CTA's memory is reused
     if (q_issued) mbar_wait(q_full, 0, p.wait_ns, no_abort);
   } else if (warp == kMmaWarp) {
@@ -273,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t kdesc0 = make_sdesc(smem_u32(sKV), 16, 1024, kSwizzle128);
       const uint64_t qdesc0 = make_sdesc(smem_u32(sQ), 16, 1024, kSwizzle128);
       const uint64_t vdesc0 =
-          make_sdesc(smem_u32(sKV) + (uint32_t)(half * C::DVH / 64) * C::KV_ATOM, C::KV_ATOM, 1024, kSwizzle128);
+          make_sdesc(smem_u32(sKV) + (uint32_t)(half * C::DVH / 64) * C::ATOM_STRIDE, C::ATOM_STRIDE, 1024, kSwizzle128);
       bool ok = nchunks == 0 || ((C::QS_ATOMS == 0 || mbar_wait(q_full, 0, p.wait_ns, ab)) &&
                                  mbar_wait(q_ready, 0, p.wait_ns, ab));
       if (!ok) fail(3);
@@ -281,22 +297,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       // landed and P V of chunk qk - kSBuf has freed its S buffer; P V of
       // chunk pv once its probabilities are written.
       int qk = 0, pv = 0;
+      // P V of chunk pv: 4 K steps of 16 keys, A = P (TMEM), B = V (MN-major);
+      // its commits free the chunk's S buffer and both ring slots
+      auto issue_pv = [&]() {
+        tc_fence_after();
+        const int s0 = (2 * pv) % kSlots, sb = pv % kSBuf;
+        const uint64_t vst = vdesc0 + (uint64_t)((s0 * C::SLOT_ATOM) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < kN / 16; ++ks) {
+          const uint64_t vdesc = vst + (uint64_t)((ks * 16 * 128) >> 4);
+          mma_bf16_ts(tmem + C::OCOL, tmem + C::SCOL + sb * kN + ks * 8, vdesc, idesc_pv,
+                      (pv > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&pv_done[sb]);
+        mma_commit(&kv_empty[s0]);
+        mma_commit(&kv_empty[s0 + 1]);
+        ++pv;
+      };
       uint64_t t_idle = 0;
       uint32_t spins = 0;
       while (ok && pv < nchunks) {
         bool progressed = false;
         if (qk < nchunks && qk < pv + kSBuf) {
-          const int st = qk % kStages, sb = qk % kSBuf;
-          if (mbar_test_wait(&kv_full[st], (qk / kStages) & 1) &&
+          const int s0 = (2 * qk) % kSlots, sb = qk % kSBuf;
+          const uint32_t par = (uint32_t)((2 * qk) / kSlots) & 1;
+          if (mbar_test_wait(&kv_full[s0], par) && mbar_test_wait(&kv_full[s0 + 1], par) &&
               (qk < kSBuf || mbar_test_wait(&pv_done[sb], ((qk / kSBuf) - 1) & 1))) {
             fence_proxy_async_smem();
             tc_fence_after();
-            const uint64_t kst = kdesc0 + (uint64_t)((st * C::STAGE) >> 4);
+            const uint64_t kst = kdesc0 + (uint64_t)((s0 * C::SLOT_ATOM) >> 4);
             const uint32_t dS = tmem + C::SCOL + sb * kN;
 #pragma unroll
             for (int ks = 0; ks < C::KSTEPS; ++ks) {
               const int d = ks * 16;
-              const uint64_t bdesc = kst + (uint64_t)(((d / 64) * C::KV_ATOM + (d % 64) * 2) >> 4);
+              const uint64_t bdesc = kst + (uint64_t)(((d / 64) * C::ATOM_STRIDE + (d % 64) * 2) >> 4);
               if (ks < C::QT_STEPS) {
                 mma_bf16_ts(dS, tmem + C::QCOL + ks * 8, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
               } else {
@@ -311,19 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (pv < qk && mbar_test_wait(&p_full[pv % kSBuf], (pv / kSBuf) & 1)) {
-          tc_fence_after();
-          const int st = pv % kStages, sb = pv % kSBuf;
-          const uint64_t vst = vdesc0 + (uint64_t)((st * C::STAGE) >> 4);
-#pragma unroll
-          for (int ks = 0; ks < kN / 16; ++ks) {
-            // A = P rows (TMEM, 8 columns = 16 BF16 keys per step), B = V (MN-major)
-            const uint64_t vdesc = vst + (uint64_t)((ks * 16 * 128) >> 4);
-            mma_bf16_ts(tmem + C::OCOL, tmem + C::SCOL + sb * kN + ks * 8, vdesc, idesc_pv,
-                        (pv > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&pv_done[sb]);
-          mma_commit(&kv_empty[st]);
-          ++pv;
+          issue_pv();
           progressed = true;
         }
         if (progressed) {
@@ -335,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pv < qk)
           mbar_try_wait_hint(&p_full[pv % kSBuf], (pv / kSBuf) & 1, 200);
         else
-          mbar_try_wait_hint(&kv_full[qk % kStages], (qk / kStages) & 1, 200);
+          mbar_try_wait_hint(&kv_full[(2 * qk) % kSlots], (uint32_t)((2 * qk) / kSlots) & 1, 200);
         if (++spins == 1) t_idle = global_ns();
         if ((spins & 1023u) == 0u) {
           if (*abort_flag != 0) { ok = false; break; }
@@ -350,8 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
       // drain: the last arrivals of each commit barrier are not always waited
       // by their consumers; make sure they have landed before the CTA exits
-      for (int i = max(0, pv - kStages); i < pv; ++i)
-        mbar_wait(&kv_empty[i % kStages], (i / kStages) & 1, p.wait_ns, no_abort);
+      for (int c = max(0, 2 * pv - kSlots); c < 2 * pv; ++c)
+        mbar_wait(&kv_empty[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
       for (int i = max(0, pv - kSBuf); i < pv; ++i)
         mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
       for (int i = max(0, qk - kSBuf); i < qk; ++i)
@@ -359,14 +381,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + output
+    // two warps per TMEM lane quarter: side 0 takes keys 0-31 of every chunk
+    // and value columns 0-127 of this CTA's half, side 1 keys 32-63 and value
+    // columns 128-255; both derive the same running maximum from the
+    // exchanged partial maxima
+    const int side = (warp - kFirstSoftmaxWarp) >> 2;
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;              // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const bool head_ok = row_ok && h < p.H;
-    // Q dims [0, QT_DIMS) of row h into TMEM as BF16 pairs (zeros past H)
+    constexpr int OHALF = C::DVH / 2;               // output columns per side
+    // Q dims [0, QT_DIMS) of row h into TMEM as BF16 pairs (zeros past H);
+    // side s writes the 64-dim blocks s, s + 2, ...
     {
       const uint16_t* qrow = p.q + ((size_t)(head_ok ? row : 0) * p.H + (head_ok ? h : 0)) * DK;
-      for (int qb = 0; qb < C::QT_BLOCKS; ++qb) {
+      for (int qb = side; qb < C::QT_BLOCKS; qb += 2) {
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -386,29 +415,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(q_ready);
     }
     const float sc = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f;              // l: this side's share of the row sum
     bool ok = true;
     for (int j = 0; j < nchunks && ok; ++j) {
-      const int sb = j % kSBuf, st = j % kStages;
-      // 1. logits of this chunk and its valid slots
+      const int sb = j % kSBuf, s0 = (2 * j) % kSlots;
+      const uint32_t kpar = (uint32_t)((2 * j) / kSlots) & 1;
+      // 1. this side's 32 logits and valid keys
       if (!wwait(&s_full[sb], (j / kSBuf) & 1)) { fail(6); ok = false; break; }
-      if (!wwait(&kv_full[st], (j / kStages) & 1)) { fail(7); ok = false; break; }
-      const uint32_t mask = sMask[st];
+      if (!wwait(&kv_full[s0 + side], kpar)) { fail(7); ok = false; break; }
+      const uint32_t mask = sMask[s0 + side];
       tc_fence_after();
       const uint32_t saddr = tmem + lane_addr + C::SCOL + sb * kN;
-      uint32_t sr[kN];
-      tmem_ld32(saddr, sr);
+      uint32_t sr[32];
+      tmem_ld32(saddr + side * 32, sr);
       tmem_wait_ld_dep(sr);
-      // 2. running maximum (log2 units; the scale is positive)
-      float mraw = -INFINITY;
+      float pm = -INFINITY;
       if (mask == 0xffffffffu) {
 #pragma unroll
-        for (int q = 0; q < kN; ++q) mraw = fmaxf(mraw, __uint_as_float(sr[q]));
+        for (int q = 0; q < 32; ++q) pm = fmaxf(pm, __uint_as_float(sr[q]));
       } else {
 #pragma unroll
-        for (int q = 0; q < kN; ++q)
-          if ((mask >> q) & 1u) mraw = fmaxf(mraw, __uint_as_float(sr[q]));
+        for (int q = 0; q < 32; ++q)
+          if ((mask >> q) & 1u) pm = fmaxf(pm, __uint_as_float(sr[q]));
       }
+      // 2. exchange the partial maxima with the other side of this quarter
+      float* xm = sXM + sb * 256;
+      xm[side * 128 + h] = pm;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mx_bar[sb * 4 + quarter]);
+      if (!wwait(&mx_bar[sb * 4 + quarter], (j / kSBuf) & 1)) { fail(10); ok = false; break; }
+      tc_fence_after();  // the other side's logits are read before P overwrites them
+      const float mraw = fmaxf(pm, xm[(side ^ 1) * 128 + h]);
       const float mc = mraw * sc;
       float alpha = 1.f;
       bool rescale = false;
@@ -419,43 +457,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_used = mc;
         rescale = true;
       }
-      // 3. rescale the output accumulator when the maximum moved (warp-wide),
-      //    once the previous P V has landed in it
+      // 3. rescale this side's output columns when the maximum moved, once
+      //    the previous P V has landed
       if (__any_sync(0xffffffffu, rescale)) {
         if (j >= 1 && !wwait(&pv_done[(j - 1) % kSBuf], ((j - 1) / kSBuf) & 1)) { fail(8); ok = false; break; }
         tc_fence_after();
-        for (int c = 0; c < C::DVH / 32; ++c) {
+        for (int c = 0; c < OHALF / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_addr + C::OCOL + c * 32, o);
+          const uint32_t oaddr = tmem + lane_addr + C::OCOL + side * OHALF + c * 32;
+          tmem_ld32(oaddr, o);
           tmem_wait_ld_dep(o);
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(tmem + lane_addr + C::OCOL + c * 32, o);
+          tmem_st32(oaddr, o);
         }
         tmem_wait_st();
       }
-      // 4. probabilities as BF16 pairs over the first kN/2 columns of the S
-      //    buffer (already read above)
+      // 4. probabilities of this side's keys as BF16 pairs over P columns
+      //    [16 side, 16 side + 16) of the S buffer (side 0's logits there
+      //    were read before its maximum was published)
       float rs = 0.f;
-      uint32_t pk[kN / 2];
-      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      uint32_t pk[16];
+      if (m_used == -INFINITY) {
 #pragma unroll
-      for (int q = 0; q < kN / 2; ++q) {
-        float e0 = exp2f(fmaf(__uint_as_float(sr[2 * q]), sc, neg_m));
-        float e1 = exp2f(fmaf(__uint_as_float(sr[2 * q + 1]), sc, neg_m));
-        if (!((mask >> (2 * q)) & 1u) || m_used == -INFINITY) e0 = 0.f;
-        if (!((mask >> (2 * q + 1)) & 1u) || m_used == -INFINITY) e1 = 0.f;
-        rs += e0 + e1;
-        pk[q] = pack_bf16x2(e0, e1);
+        for (int q = 0; q < 16; ++q) pk[q] = 0u;
+      } else {
+        const float neg_m = -m_used;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float e0 = ex2_approx(fmaf(__uint_as_float(sr[2 * q]), sc, neg_m));
+          float e1 = ex2_approx(fmaf(__uint_as_float(sr[2 * q + 1]), sc, neg_m));
+          if (mask != 0xffffffffu) {
+            if (!((mask >> (2 * q)) & 1u)) e0 = 0.f;
+            if (!((mask >> (2 * q + 1)) & 1u)) e1 = 0.f;
+          }
+          rs += e0 + e1;
+          pk[q] = pack_bf16x2(e0, e1);
+        }
       }
-      tmem_st16(saddr, pk);
+      tmem_st16(saddr + side * 16, pk);
       tmem_wait_st();
       l = l * alpha + rs;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    // 5. output
+    // 5. output: combine the two partial row sums, then each side writes its
+    //    value columns
+    if (ok && nchunks > 0) {
+      float* xl = sXM + (nchunks % kSBuf) * 256;    // buffer of chunk nchunks - 2, no longer read
+      xl[side * 128 + h] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lx_bar[quarter]);
+      if (!wwait(&lx_bar[quarter], 0)) {
+        fail(11);
+        ok = false;
+      } else {
+        l += xl[(side ^ 1) * 128 + h];
+      }
+    }
     if (ok && nchunks > 0 && !wwait(&pv_done[(nchunks - 1) % kSBuf], ((nchunks - 1) / kSBuf) & 1)) {
       fail(9);
       ok = false;
@@ -464,10 +524,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m_used + log2f(l) : -INFINITY;
-      const int vlo = half * C::DVH;
-      for (int c = 0; c < C::DVH / 32; ++c) {
+      const int vlo = half * C::DVH + side * OHALF;
+      for (int c = 0; c < OHALF / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_addr + C::OCOL + c * 32, o);
+        tmem_ld32(tmem + lane_addr + C::OCOL + side * OHALF + c * 32, o);
         tmem_wait_ld_dep(o);
         if (!head_ok) continue;
         if (p.nsplit == 1) {
@@ -490,14 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __uint_as_float(o[4 * g + 2]) * inv, __uint_as_float(o[4 * g + 3]) * inv);
         }
       }
-      if (half == 0 && head_ok) {
+      if (half == 0 && side == 0 && head_ok) {
         if (p.nsplit == 1) {
           if (p.lse != nullptr) p.lse[(size_t)row * p.H + h] = lse2 * 0.6931471805599453f;
         } else {
           p.part_lse[((size_t)row * p.nsplit + split) * p.H + h] = lse2;
         }
       }
-    } else if (ok && head_ok && half == 0) {
+    } else if (ok && head_ok && half == 0 && side == 0) {
       // no selected slots in this split: empty result
       if (p.nsplit > 1) p.part_lse[((size_t)row * p.nsplit + split) * p.H + h] = -INFINITY;
     }
