@@ -41,9 +41,17 @@ constexpr int kKC = 32;        // key tiles per work item (at most; fewer when i
 constexpr int kStages = 4;     // depth of the k_I ring
 constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * kNSub = 512 columns)
 static_assert((kNAcc & (kNAcc - 1)) == 0, "accumulator index is taken with a mask");
-constexpr int kEpiGroups = 3;   // epilogue groups of four warps
-constexpr int kEpiThreads = 128 * kEpiGroups;
-constexpr int kThreads = 64 + kEpiThreads;
+// Key tiles per accumulator group: with many heads (HI >= 32) two
+// consecutive key tiles share one pass of the epilogue over a sub-tile, so
+// every head-weight load from shared memory serves two accumulators.
+template <int HI>
+struct EpiCfg {
+  static constexpr int G = HI >= 32 ? 2 : 1;       // key tiles per group
+  static constexpr int NSLOT = kNAcc / G;          // accumulator groups in flight
+  static constexpr int NGRP = G == 2 ? 2 : 3;      // epilogue groups of four warps
+  static constexpr int EPI_THREADS = 128 * NGRP;
+  static constexpr int THREADS = 64 + EPI_THREADS;
+};
 
 struct IdxParams {
   const float* w;
@@ -129,7 +137,7 @@ __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, 
 }
 
 template <int DI, int HI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                       IdxParams p) {
   using L = Layout<DI>;
@@ -165,8 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], 4);  // one arrive per epilogue warp of the owning group
     }
     mbar_init(mma_done, 1);
-    mbar_init(&w_ready[0], kEpiThreads);
-    mbar_init(&w_ready[1], kEpiThreads);
+    mbar_init(&w_ready[0], EpiCfg<HI>::EPI_THREADS);
+    mbar_init(&w_ready[1], EpiCfg<HI>::EPI_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -228,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc(kFmtE4M3, kFmtE4M3, 0, 0, kBM, kNSub);
+      using E = EpiCfg<HI>;
       uint32_t a_cnt = 0, items = 0, u = 0;
       // descriptors built once; a stage or sub-tile only adds its offset >> 4
       const uint64_t adesc0 = make_sdesc(smem_u32(sA), 16, L::kSBO, L::kSwizzleLayout);
@@ -237,28 +246,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++items;
         const int nsub = item_nsub<HI>(p, it);
         const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
-        for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
-          const int st = a_cnt % kStages;
-          if (!mbar_wait(&a_full[st], (a_cnt / kStages) & 1, p.wait_ns, ab)) { fail(4); return false; }
+        for (int kt = kt0; kt < kt1; kt += E::G) {
+          // key tiles kt .. kt + ng - 1 of this group, each in its ring stage
+          const int ng = min(E::G, kt1 - kt);
+          uint64_t adesc[E::G];
+#pragma unroll
+          for (int g = 0; g < E::G; ++g) {
+            if (g >= ng) break;
+            const uint32_t c = a_cnt + (uint32_t)g;
+            const int st = c % kStages;
+            if (!mbar_wait(&a_full[st], (c / kStages) & 1, p.wait_ns, ab)) { fail(4); return false; }
+            adesc[g] = adesc0 + (uint64_t)((st * L::kABytes) >> 4);
+          }
           tc_fence_after();
-          const uint64_t adesc = adesc0 + (uint64_t)((st * L::kABytes) >> 4);
+          // the first active sub-tile of kt also covers kt + 1 (later keys
+          // need later queries); masked pairs are computed and dropped
           for (int j = first_active<HI>(p, it, kt, nsub); j < nsub; ++j) {
-            const int acc = u & (kNAcc - 1);
-            if (!mbar_test_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1) &&
-                !mbar_wait(&acc_empty[acc], ((u / kNAcc) & 1) ^ 1, p.wait_ns, ab)) {
+            const int slot = u % E::NSLOT;
+            if (!mbar_test_wait(&acc_empty[slot], ((u / E::NSLOT) & 1) ^ 1) &&
+                !mbar_wait(&acc_empty[slot], ((u / E::NSLOT) & 1) ^ 1, p.wait_ns, ab)) {
               fail(5);
               return false;
             }
             tc_fence_after();
             const uint64_t bdesc = bdesc0 + (uint64_t)((j * L::kBSubBytes) >> 4);
-            const uint32_t dacc = tmem_base + acc * kNSub;
 #pragma unroll
-            for (int ks = 0; ks < DI / 32; ++ks)
-              mma_f8(dacc, adesc + 2 * ks, bdesc + 2 * ks, idesc, ks > 0 ? 1u : 0u);
-            mma_commit(&acc_full[acc]);
+            for (int g = 0; g < E::G; ++g) {
+              if (g >= ng) break;
+              const uint32_t dacc = tmem_base + (slot * E::G + g) * kNSub;
+#pragma unroll
+              for (int ks = 0; ks < DI / 32; ++ks)
+                mma_f8(dacc, adesc[g] + 2 * ks, bdesc + 2 * ks, idesc, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&acc_full[slot]);
             ++u;
           }
-          mma_commit(&a_empty[st]);
+#pragma unroll
+          for (int g = 0; g < E::G; ++g) {
+            if (g >= ng) break;
+            mma_commit(&a_empty[(a_cnt + (uint32_t)g) % kStages]);
+          }
+          a_cnt += (uint32_t)ng;
         }
         mma_commit(b_empty);
         return true;
@@ -268,16 +296,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    const int ew = warp - 2;             // 0 .. 4 * kEpiGroups - 1
-    const int grp = ew >> 2;             // drains sub-tiles u with u % kEpiGroups == grp
+    using E = EpiCfg<HI>;
+    const int ew = warp - 2;             // 0 .. 4 * NGRP - 1
+    const int grp = ew >> 2;             // drains groups u with u % NGRP == grp
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
-    const int r = quarter * 32 + lane;   // key row within the tile
-    const int etid = threadIdx.x - 64;   // 0..255
+    const int r = quarter * 32 + lane;   // key row within a tile
+    const int etid = threadIdx.x - 64;
     uint32_t u = 0, items = 0;
     for_each_item<HI>(p, [&](const Item& it) {
       // per-item head weights  wM[(query, head)] = w * q_scale  (0 past the end)
       float* wbuf = sW + (items & 1) * L::kWFloats;
-      for (int x = etid; x < p.nb * kNSub; x += kEpiThreads) {
+      for (int x = etid; x < p.nb * kNSub; x += E::EPI_THREADS) {
         const int t = it.t0 + x / HI;
         float v = 0.f;
         if (t < it.tend) {
@@ -291,76 +320,95 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++items;
       const int nsub = item_nsub<HI>(p, it);
       const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
-      for (int kt = kt0; kt < kt1; ++kt) {
-        const int s = kt * kBM + r;
-        const float ks = s < p.S ? p.k_scale[(size_t)it.b * p.S + s] : 0.f;
+      for (int kt = kt0; kt < kt1; kt += E::G) {
+        const int ng = min(E::G, kt1 - kt);
+        int sg[E::G];
+        float ksg[E::G];
+#pragma unroll
+        for (int g = 0; g < E::G; ++g) {
+          sg[g] = (kt + g) * kBM + r;
+          ksg[g] = (g < ng && sg[g] < p.S) ? p.k_scale[(size_t)it.b * p.S + sg[g]] : 0.f;
+        }
         const int jlo = first_active<HI>(p, it, kt, nsub);
         const uint32_t u0 = u;
         u += (uint32_t)(nsub - jlo);
-        // this group's sub-tiles of the tile: my = u0 + (j - jlo) == grp (mod kEpiGroups)
-        const int skip = (int)((grp + kEpiGroups - (int)(u0 % kEpiGroups)) % kEpiGroups);
-        for (int j = jlo + skip; j < nsub; j += kEpiGroups) {
+        // this group's sub-tiles: my = u0 + (j - jlo) == grp (mod NGRP)
+        const int skip = (int)((grp + E::NGRP - (int)(u0 % E::NGRP)) % E::NGRP);
+        for (int j = jlo + skip; j < nsub; j += E::NGRP) {
           const uint32_t my = u0 + (uint32_t)(j - jlo);
-          const int acc = my & (kNAcc - 1);
-          const bool got = mbar_wait(&acc_full[acc], (my / kNAcc) & 1, p.wait_ns, ab);
+          const int slot = my % E::NSLOT;
+          const bool got = mbar_wait(&acc_full[slot], (my / E::NSLOT) & 1, p.wait_ns, ab);
           if (!__all_sync(0xffffffffu, got)) { fail(6); return false; }
           tc_fence_after();
-          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kNSub;
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot * E::G * kNSub;
           const float* wq = wbuf + j * kNSub;
-          // w * ReLU(x) summed over the heads of each query: four independent
-          // packed-pair partial sums per query keep the FMA chains short
+          // w * ReLU(x) summed over the heads of each query, for each key tile
+          // of the group; four independent packed-pair partial sums per
+          // (tile, query) keep the FMA chains short
           constexpr int NP = HI >= 8 ? 4 : 2;
-          float2 part[QPS][NP];
+          constexpr int CW = 16;                      // TMEM columns per load
+          float2 part[E::G][QPS][NP];
 #pragma unroll
-          for (int q = 0; q < QPS; ++q)
+          for (int g = 0; g < E::G; ++g)
 #pragma unroll
-            for (int i = 0; i < NP; ++i) part[q][i] = make_float2(0.f, 0.f);
-          uint32_t v[2][32];
-          tmem_ld32(taddr, v[0]);
-          tmem_wait_ld_dep(v[0]);
+            for (int q = 0; q < QPS; ++q)
 #pragma unroll
-          for (int c = 0; c < kNSub / 32; ++c) {
-            if (c + 1 < kNSub / 32) {
-              tmem_ld32(taddr + (c + 1) * 32, v[(c + 1) & 1]);
+              for (int i = 0; i < NP; ++i) part[g][q][i] = make_float2(0.f, 0.f);
+          uint32_t v[2][E::G][CW];
+#pragma unroll
+          for (int g = 0; g < E::G; ++g) tmem_ld16(taddr + g * kNSub, v[0][g]);
+#pragma unroll
+          for (int g = 0; g < E::G; ++g) tmem_wait_ld_dep(v[0][g]);
+#pragma unroll
+          for (int c = 0; c < kNSub / CW; ++c) {
+            if (c + 1 < kNSub / CW) {
+#pragma unroll
+              for (int g = 0; g < E::G; ++g) tmem_ld16(taddr + g * kNSub + (c + 1) * CW, v[(c + 1) & 1][g]);
             } else {
-              // every column of this accumulator is in registers: hand it back
+              // every column of the group's accumulators is in registers
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[acc]);
+              if (lane == 0) mbar_arrive(&acc_empty[slot]);
             }
 #pragma unroll
-            for (int e = 0; e < 32; e += 2 * NP) {
-              const int q = (c * 32 + e) / HI;
+            for (int e = 0; e < CW; e += 2 * NP) {
+              const int q = (c * CW + e) / HI;
 #pragma unroll
               for (int i = 0; i < NP; i += 2) {
-                const float4 w4 = *reinterpret_cast<const float4*>(wq + c * 32 + e + 2 * i);
-                const uint32_t* x = &v[c & 1][e + 2 * i];
-                const float2 r0 = make_float2(fmaxf(__uint_as_float(x[0]), 0.f), fmaxf(__uint_as_float(x[1]), 0.f));
-                const float2 r1 = make_float2(fmaxf(__uint_as_float(x[2]), 0.f), fmaxf(__uint_as_float(x[3]), 0.f));
-                part[q][i] = __ffma2_rn(make_float2(w4.x, w4.y), r0, part[q][i]);
-                part[q][i + 1] = __ffma2_rn(make_float2(w4.z, w4.w), r1, part[q][i + 1]);
+                const float4 w4 = *reinterpret_cast<const float4*>(wq + c * CW + e + 2 * i);
+#pragma unroll
+                for (int g = 0; g < E::G; ++g) {
+                  const uint32_t* x = &v[c & 1][g][e + 2 * i];
+                  const float2 r0 = make_float2(fmaxf(__uint_as_float(x[0]), 0.f), fmaxf(__uint_as_float(x[1]), 0.f));
+                  const float2 r1 = make_float2(fmaxf(__uint_as_float(x[2]), 0.f), fmaxf(__uint_as_float(x[3]), 0.f));
+                  part[g][q][i] = __ffma2_rn(make_float2(w4.x, w4.y), r0, part[g][q][i]);
+                  part[g][q][i + 1] = __ffma2_rn(make_float2(w4.z, w4.w), r1, part[g][q][i + 1]);
+                }
               }
             }
-            if (c + 1 < kNSub / 32) tmem_wait_ld_dep(v[(c + 1) & 1]);
-          }
-          float accq[QPS];
+            if (c + 1 < kNSub / CW) {
 #pragma unroll
-          for (int q = 0; q < QPS; ++q) {
-            float a = 0.f;
-#pragma unroll
-            for (int i = 0; i < NP; ++i) a += part[q][i].x + part[q][i].y;
-            accq[q] = a;
+              for (int g = 0; g < E::G; ++g) tmem_wait_ld_dep(v[(c + 1) & 1][g]);
+            }
           }
 #pragma unroll
-          for (int q = 0; q < QPS; ++q) {
-            const int t = it.t0 + j * QPS + q;
-            if (t < it.tend && s <= p.S - p.T + t) {
-              // self-check: the score slot lies inside this launch's tile
-              const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
-              if (ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld)
-                p.scores[ri * p.ld + s] = accq[q] * ks;
-              else
-                report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
+          for (int g = 0; g < E::G; ++g) {
+            if (g >= ng) break;
+            const int s = sg[g];
+#pragma unroll
+            for (int q = 0; q < QPS; ++q) {
+              float a = 0.f;
+#pragma unroll
+              for (int i = 0; i < NP; ++i) a += part[g][q][i].x + part[g][q][i].y;
+              const int t = it.t0 + j * QPS + q;
+              if (t < it.tend && s <= p.S - p.T + t) {
+                // self-check: the score slot lies inside this launch's tile
+                const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
+                if (ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld)
+                  p.scores[ri * p.ld + s] = a * ksg[g];
+                else
+                  report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
+              }
             }
           }
         }
@@ -429,7 +477,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<DI, HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::kAlloc);
   if (e != cudaSuccess) return e;
-  indexer_tc_kernel<DI, HI><<<grid, kThreads, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
+  indexer_tc_kernel<DI, HI><<<grid, EpiCfg<HI>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
   note_launches(1);
   return cudaGetLastError();
 }
