@@ -200,7 +200,11 @@ class DsaRunner:
         self.ws = dsa.alloc_workspace(self.shape)
         self.outs = dsa.alloc_outputs(wl)
         self.ld = (wl.S + 63) // 64 * 64
-        self.scores = self.ws[: wl.B * self.rows_per_block() * self.ld * 4].view(torch.float32).view(-1, self.ld)
+        nscore = wl.B * self.rows_per_block() * self.ld * 4
+        self.scores = self.ws[:nscore].view(torch.float32).view(-1, self.ld)
+        # the top-k's scratch (histograms of the split path for few long
+        # rows) follows the scores, 256-byte aligned, as in dsa_forward
+        self.topk_ws = self.ws[(nscore + 255) // 256 * 256:]
         self.stream = torch.cuda.current_stream()
 
     def rows_per_block(self):
@@ -225,7 +229,7 @@ class DsaRunner:
             e0 = mark()
             d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, self.scores)
             e1 = mark()
-            d.topk(self.shape, self.scores, q0, cnt, o.idx)
+            d.topk(self.shape, self.scores, q0, cnt, o.idx, self.topk_ws)
             e2 = mark()
             if ev is not None:
                 ev.append(("indexer", e0, e1))

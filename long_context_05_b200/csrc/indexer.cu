@@ -76,7 +76,7 @@ struct Layout {
   static constexpr int kWOff = kAOff + kStages * kABytes;            // wM, two item buffers
   static constexpr int kWFloats = kMaxNB * kNSub;
   static constexpr int kBarOff = kWOff + 2 * kWFloats * 4;
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 * kNAcc + 1 + 2;
+  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNAcc + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
@@ -150,9 +150,9 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + kStages;
-  uint64_t* b_full = bars + 2 * kStages;
-  uint64_t* b_empty = b_full + 1;
-  uint64_t* acc_full = b_full + 2;
+  uint64_t* b_full = bars + 2 * kStages;       // [2] B buffer loaded (TMA)
+  uint64_t* b_empty = b_full + 2;              // [2] B buffer free (MMA commit)
+  uint64_t* acc_full = b_empty + 2;
   uint64_t* acc_empty = acc_full + kNAcc;
   uint64_t* mma_done = acc_empty + kNAcc;
   uint64_t* w_ready = mma_done + 1;  // [2]: epilogue threads finished filling wM buffer
@@ -160,14 +160,21 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // With at most half of the B sub-tiles in use (few queries per item, as in
+  // decode), the B region holds two item buffers, so the next item's B and
+  // its first key tiles load while the current item's MMAs run.
+  const int nbbuf = p.nb * 2 <= kMaxNB ? 2 : 1;
+  constexpr int kBBufBytes = kMaxNB / 2 * L::kBSubBytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&a_full[i], 1);
       mbar_init(&a_empty[i], 1);
     }
-    mbar_init(b_full, 1);
-    mbar_init(b_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
     for (int i = 0; i < kNAcc; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);  // one arrive per epilogue warp of the owning group
@@ -205,13 +212,15 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       for (int i = 0; i < kStages; ++i) issued[i] = false;
       bool ok = true;
       for_each_item<HI>(p, [&](const Item& it) {
-        if (!mbar_wait(b_empty, (items & 1) ^ 1, p.wait_ns, ab)) { fail(1); ok = false; return false; }
+        const int bb = nbbuf == 2 ? (int)(items & 1) : 0;
+        const uint32_t use = nbbuf == 2 ? items >> 1 : items;
+        if (!mbar_wait(&b_empty[bb], (use & 1) ^ 1, p.wait_ns, ab)) { fail(1); ok = false; return false; }
         int nsub = 0;
         for (int j = 0; j < p.nb; ++j)
           if (it.t0 + j * QPS < it.tend) nsub = j + 1;
-        mbar_arrive_expect_tx(b_full, nsub * L::kBSubBytes);
+        mbar_arrive_expect_tx(&b_full[bb], nsub * L::kBSubBytes);
         for (int j = 0; j < nsub; ++j)
-          tma_load_2d(sB + j * L::kBSubBytes, &tm_q, b_full, 0, (it.b * p.T + it.t0 + j * QPS) * HI);
+          tma_load_2d(sB + bb * kBBufBytes + j * L::kBSubBytes, &tm_q, &b_full[bb], 0, (it.b * p.T + it.t0 + j * QPS) * HI);
         ++items;
         const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
         for (int kt = kt0; kt < kt1; ++kt, ++a_cnt) {
@@ -229,7 +238,11 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       // let every load this CTA started land before it exits
       for (int st = 0; st < kStages; ++st)
         if (issued[st]) mbar_wait(&a_full[st], last_phase[st], p.wait_ns, no_abort);
-      if (items > 0) mbar_wait(b_full, (items - 1) & 1, p.wait_ns, no_abort);
+      for (uint32_t i = items > 2 ? items - 2 : 0; i < items; ++i) {
+        const int bb = nbbuf == 2 ? (int)(i & 1) : 0;
+        const uint32_t use = nbbuf == 2 ? i >> 1 : i;
+        if (nbbuf == 2 || i + 1 == items) mbar_wait(&b_full[bb], use & 1, p.wait_ns, no_abort);
+      }
       (void)ok;
     }
   } else if (warp == 1) {
@@ -242,8 +255,11 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       const uint64_t adesc0 = make_sdesc(smem_u32(sA), 16, L::kSBO, L::kSwizzleLayout);
       const uint64_t bdesc0 = make_sdesc(smem_u32(sB), 16, L::kSBO, L::kSwizzleLayout);
       for_each_item<HI>(p, [&](const Item& it) {
-        if (!mbar_wait(b_full, items & 1, p.wait_ns, ab)) { fail(3); return false; }
+        const int bb = nbbuf == 2 ? (int)(items & 1) : 0;
+        const uint32_t use = nbbuf == 2 ? items >> 1 : items;
+        if (!mbar_wait(&b_full[bb], use & 1, p.wait_ns, ab)) { fail(3); return false; }
         ++items;
+        const uint64_t bdesc_it = bdesc0 + (uint64_t)((bb * kBBufBytes) >> 4);
         const int nsub = item_nsub<HI>(p, it);
         const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
         for (int kt = kt0; kt < kt1; kt += E::G) {
@@ -269,7 +285,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
               return false;
             }
             tc_fence_after();
-            const uint64_t bdesc = bdesc0 + (uint64_t)((j * L::kBSubBytes) >> 4);
+            const uint64_t bdesc = bdesc_it + (uint64_t)((j * L::kBSubBytes) >> 4);
 #pragma unroll
             for (int g = 0; g < E::G; ++g) {
               if (g >= ng) break;
@@ -288,7 +304,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           }
           a_cnt += (uint32_t)ng;
         }
-        mma_commit(b_empty);
+        mma_commit(&b_empty[bb]);
         return true;
       });
       mma_commit(mma_done);

@@ -21,8 +21,12 @@
 //      complement of the index picks them).
 // If bin B holds more candidates than shared memory takes, steps 2-3 run as
 // radix passes over the row itself and a final pass in index order.
-// Decode rows (few, long) are split over several blocks for steps 1-2, with
-// the histogram and the candidates gathered in the caller's workspace.
+// Decode rows (few, long) are split over several blocks for steps 1-2: the
+// blocks of a row add their histograms in the caller's workspace, then each
+// block finds bin B from the row's histogram and, over its own segment,
+// writes the keys above B to the output and appends bin B's keys to a
+// per-row candidate list in the workspace (warp-aggregated atomics); one
+// block per row finishes step 3 on that list.
 #include "internal.h"
 
 namespace dsa {
@@ -34,6 +38,13 @@ constexpr int kBins = 2048;           // top 11 bits
 constexpr int kBinShift = 21;
 constexpr int kCap = 8192;            // candidates held in shared memory
 constexpr int kSegBlocks = 16;        // blocks per row in the split (decode) path
+// Split-path workspace per row, in 32-bit words: histogram | counters (keys
+// written, candidates) | candidate keys | candidate indices.
+constexpr int kWsHist = 0;
+constexpr int kWsCtr = kBins;
+constexpr int kWsKeys = kBins + 4;
+constexpr int kWsIdx = kWsKeys + kCap;
+constexpr int kWsRowWords = kWsIdx + kCap;
 
 __device__ __forceinline__ unsigned int order_key(float f) {
   unsigned int u = __float_as_uint(f);
@@ -447,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevEr
 // Workspace per row: hist[kBins] u32.  Kernel 1 adds each segment's histogram;
 // kernel 2 (one block per row) finds the bin and runs steps 2-3.
 
-__global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist) {
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist, int hstride) {
   __shared__ unsigned int hist[kBins];
   const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
   int b, t, n;
@@ -461,9 +472,127 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, 
   const int lo = seg * per, hi = min(n, lo + per);
   if (lo < hi) histogram_pass(row, lo, hi, hist);
   __syncthreads();
-  unsigned int* gh = ghist + (size_t)r * kBins;
+  unsigned int* gh = ghist + (size_t)r * hstride;
   for (int x = threadIdx.x; x < kBins; x += kThreads)
     if (hist[x]) atomicAdd(&gh[x], hist[x]);
+}
+
+// Warp-aggregated append: every lane of the warp calls this (flag may be
+// false); returns this lane's slot for a true flag (else -1).
+__device__ __forceinline__ int warp_append(bool flag, unsigned int* counter) {
+  const unsigned int bal = __ballot_sync(0xffffffffu, flag);
+  if (bal == 0u) return -1;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(bal) - 1;
+  unsigned int base = 0;
+  if (lane == leader) base = atomicAdd(counter, (unsigned int)__popc(bal));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  return flag ? (int)(base + __popc(bal & ((1u << lane) - 1u))) : -1;
+}
+
+// Split path, step 2 over one segment of a row: find bin B from the row's
+// histogram, write the keys above B, append bin B's keys to the candidates.
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
+  __shared__ unsigned int hist[kBins];
+  __shared__ unsigned int warp_tot[kWarps];
+  __shared__ unsigned int s_bin, s_above, s_total;
+  const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, r, &b, &t, &n, &row, &out);
+  const int k = a.k;
+  if (n <= k) return;
+  unsigned int* w = ws + (size_t)r * kWsRowWords;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) hist[x] = w[kWsHist + x];
+  if (threadIdx.x == 0) s_bin = 0xFFFFFFFFu;
+  __syncthreads();
+  find_bin(hist, kBins, (unsigned int)k, warp_tot, &s_bin, &s_above, &s_total);
+  const unsigned int B = s_bin;
+  if (B >= (unsigned)kBins) return;  // reported by the final kernel
+  unsigned int* cnt = w + kWsCtr;
+  unsigned int* ncand = w + kWsCtr + 1;
+  unsigned int* ck = w + kWsKeys;
+  int* ci = reinterpret_cast<int*>(w + kWsIdx);
+  const int per = ((n + kSegBlocks - 1) / kSegBlocks + 3) & ~3;
+  const int lo = seg * per, hi = min(n, lo + per);
+  if (lo >= hi) return;  // past the end of a short row
+  // every lane runs the same number of rounds (ballots need the full warp)
+  auto visit = [&](bool valid, float f, int x) {
+    const unsigned int bin = order_key(f) >> kBinShift;
+    const int po = warp_append(valid && bin > B, cnt);
+    if (po >= 0) put(out, k, po, x, err, 10);
+    const int pc = warp_append(valid && bin == B, ncand);
+    if (pc >= 0 && pc < kCap) {
+      ck[pc] = order_key(f);
+      ci[pc] = x;
+    }
+  };
+  const int n4lo = lo / 4, n4hi = hi / 4;  // lo is a multiple of 4
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  for (int base = n4lo; base < n4hi; base += 2 * kThreads) {
+    float4 v[2];
+    bool ok[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int x = base + u * kThreads + (int)threadIdx.x;
+      ok[u] = x < n4hi;
+      v[u] = ok[u] ? r4[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = 4 * (base + u * kThreads + (int)threadIdx.x);
+      visit(ok[u], v[u].x, e);
+      visit(ok[u], v[u].y, e + 1);
+      visit(ok[u], v[u].z, e + 2);
+      visit(ok[u], v[u].w, e + 3);
+    }
+  }
+  {
+    const int x = 4 * n4hi + (int)threadIdx.x;  // tail of fewer than 4 keys
+    const bool ok = x < hi;
+    visit(ok, ok ? row[x] : 0.f, x);
+  }
+}
+
+// Split path, step 3: one block per row selects from the collected
+// candidates; more candidates than shared memory holds falls back to the
+// passes over the row.
+__global__ void __launch_bounds__(kThreads, 2) topk_seg_final_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, blockIdx.x, &b, &t, &n, &row, &out);
+  const int k = a.k;
+  if (n <= k) {
+    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
+    return;
+  }
+  const unsigned int* w = ws + (size_t)blockIdx.x * kWsRowWords;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = w[kWsHist + x];
+  if (threadIdx.x == 0) sm.bin = 0xFFFFFFFFu;
+  __syncthreads();
+  find_bin(sm.hist, kBins, (unsigned int)k, sm.warp_tot, &sm.bin, &sm.above, &sm.total);
+  const unsigned int B = sm.bin, above = sm.above;
+  const unsigned int inbin = B < (unsigned)kBins ? sm.hist[B] : 0u;
+  const unsigned int written = w[kWsCtr], nc = w[kWsCtr + 1];
+  __syncthreads();
+  if (B >= (unsigned)kBins || written != above || nc != inbin || nc > (unsigned)kCap) {
+    // (the first two cannot happen with a consistent histogram; the passes
+    // over the row rewrite every slot from the start)
+    select_from_bin(row, n, k, out, B, above, inbin, sm, err);
+    return;
+  }
+  for (int i = threadIdx.x; i < (int)nc; i += kThreads) {
+    sm.ck[i] = w[kWsKeys + i];
+    sm.ci[i] = static_cast<int>(w[kWsIdx + i]);
+  }
+  if (threadIdx.x == 0) sm.cnt = (int)above;
+  __syncthreads();
+  select_candidates((int)nc, B << kBinShift, 0xFFFFFFFFu << kBinShift, kBinShift, (unsigned int)k - above, k, out,
+                    sm, err);
 }
 
 __global__ void __launch_bounds__(kThreads, 2) topk_seg_select_kernel(TopkArgs a, unsigned int* ghist, DevErr* err) {
@@ -489,13 +618,16 @@ __global__ void __launch_bounds__(kThreads, 2) topk_seg_select_kernel(TopkArgs a
   select_from_bin(row, n, k, out, B, above, inbin, sm, err);
 }
 
-__global__ void topk_zero_kernel(unsigned int* p, size_t n) {
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0u;
+// Zero the first `words` words of each of `rows` rows of `stride` words.
+__global__ void topk_zero_kernel(unsigned int* p, int rows, int stride, int words) {
+  const size_t n = (size_t)rows * words;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    p[(i / words) * stride + i % words] = 0u;
 }
 
 }  // namespace
 
-size_t topk_workspace_bytes(int rows) { return (size_t)rows * kBins * sizeof(unsigned int); }
+size_t topk_workspace_bytes(int rows) { return (size_t)rows * kWsRowWords * sizeof(unsigned int); }
 
 bool topk_uses_workspace(int rows, int S, int num_sms) { return rows * 2 < num_sms && S >= 16 * kThreads; }
 
@@ -514,14 +646,14 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
     note_launches(1);
     return cudaGetLastError();
   }
-  unsigned int* gh = static_cast<unsigned int*>(ws);
-  topk_zero_kernel<<<64, 256, 0, c.stream>>>(gh, (size_t)rows * kBins);
-  note_launches(1);
-  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, gh);
-  e = cudaFuncSetAttribute(topk_seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  unsigned int* w = static_cast<unsigned int*>(ws);
+  topk_zero_kernel<<<64, 256, 0, c.stream>>>(w, rows, kWsRowWords, kWsKeys);
+  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, kWsRowWords);
+  topk_seg_collect_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, c.err);
+  e = cudaFuncSetAttribute(topk_seg_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_seg_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, gh, c.err);
-  note_launches(2);
+  topk_seg_final_kernel<<<rows, kThreads, smem, c.stream>>>(a, w, c.err);
+  note_launches(4);
   return cudaGetLastError();
 }
 
@@ -534,8 +666,8 @@ namespace dsa {
 cudaError_t launch_topk_split_into(const LaunchCtx& c, const TopkArgs& a, unsigned int* hist) {
   const int rows = a.B * a.q_count;
   if (rows <= 0) return cudaSuccess;
-  topk_zero_kernel<<<64, 256, 0, c.stream>>>(hist, (size_t)rows * kBins);
-  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, hist);
+  topk_zero_kernel<<<64, 256, 0, c.stream>>>(hist, rows, kBins, kBins);
+  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, hist, kBins);
   const size_t smem = sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(topk_seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
