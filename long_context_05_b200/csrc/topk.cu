@@ -25,8 +25,9 @@
 // blocks of a row add their histograms in the caller's workspace, then each
 // block finds bin B from the row's histogram and, over its own segment,
 // writes the keys above B to the output and appends bin B's keys to a
-// per-row candidate list in the workspace (warp-aggregated atomics); one
-// block per row finishes step 3 on that list.
+// per-row candidate list in the workspace (a block scan of the per-thread
+// counts, then one global atomic per list and block); one block per row
+// finishes step 3 on that list.
 #include "internal.h"
 
 namespace dsa {
@@ -477,19 +478,6 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, 
     if (hist[x]) atomicAdd(&gh[x], hist[x]);
 }
 
-// Warp-aggregated append: every lane of the warp calls this (flag may be
-// false); returns this lane's slot for a true flag (else -1).
-__device__ __forceinline__ int warp_append(bool flag, unsigned int* counter) {
-  const unsigned int bal = __ballot_sync(0xffffffffu, flag);
-  if (bal == 0u) return -1;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(bal) - 1;
-  unsigned int base = 0;
-  if (lane == leader) base = atomicAdd(counter, (unsigned int)__popc(bal));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  return flag ? (int)(base + __popc(bal & ((1u << lane) - 1u))) : -1;
-}
-
 // Split path, step 2 over one segment of a row: find bin B from the row's
 // histogram, write the keys above B, append bin B's keys to the candidates.
 __global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
@@ -517,41 +505,73 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs 
   const int per = ((n + kSegBlocks - 1) / kSegBlocks + 3) & ~3;
   const int lo = seg * per, hi = min(n, lo + per);
   if (lo >= hi) return;  // past the end of a short row
-  // every lane runs the same number of rounds (ballots need the full warp)
-  auto visit = [&](bool valid, float f, int x) {
-    const unsigned int bin = order_key(f) >> kBinShift;
-    const int po = warp_append(valid && bin > B, cnt);
-    if (po >= 0) put(out, k, po, x, err, 10);
-    const int pc = warp_append(valid && bin == B, ncand);
-    if (pc >= 0 && pc < kCap) {
-      ck[pc] = order_key(f);
-      ci[pc] = x;
-    }
-  };
-  const int n4lo = lo / 4, n4hi = hi / 4;  // lo is a multiple of 4
+  // Rounds of eight keys per thread (two 16-byte loads), the same number for
+  // every thread: each round counts its hits per thread, one block scan gives
+  // every thread its offsets, and one global atomic per list reserves the
+  // block's range.
+  __shared__ unsigned int s_base_out, s_base_cand;
   const float4* r4 = reinterpret_cast<const float4*>(row);
-  for (int base = n4lo; base < n4hi; base += 2 * kThreads) {
-    float4 v[2];
-    bool ok[2];
+  const int n4lo = lo / 4, n4hi = hi / 4;  // lo is a multiple of 4
+  const int tail = hi - 4 * n4hi;          // fewer than 4 keys after the last 16-byte load
+  const int rounds = (n4hi - n4lo + 2 * kThreads - 1) / (2 * kThreads) + (tail > 0 ? 1 : 0);
+  for (int rd = 0; rd < rounds; ++rd) {
+    float f[8];
+    int x[8];
+    bool ok[8];
+    const int base = n4lo + rd * 2 * kThreads;
+    if (base < n4hi) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int x = base + u * kThreads + (int)threadIdx.x;
-      ok[u] = x < n4hi;
-      v[u] = ok[u] ? r4[x] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+      for (int u = 0; u < 2; ++u) {
+        const int i4 = base + u * kThreads + (int)threadIdx.x;
+        const bool v = i4 < n4hi;
+        const float4 q = v ? r4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        f[4 * u] = q.x; f[4 * u + 1] = q.y; f[4 * u + 2] = q.z; f[4 * u + 3] = q.w;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int e = 4 * (base + u * kThreads + (int)threadIdx.x);
-      visit(ok[u], v[u].x, e);
-      visit(ok[u], v[u].y, e + 1);
-      visit(ok[u], v[u].z, e + 2);
-      visit(ok[u], v[u].w, e + 3);
+        for (int e = 0; e < 4; ++e) {
+          x[4 * u + e] = 4 * i4 + e;
+          ok[4 * u + e] = v;
+        }
+      }
+    } else {  // the last round takes the tail keys, one per thread
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ok[e] = e == 0 && (int)threadIdx.x < tail;
+        x[e] = 4 * n4hi + (int)threadIdx.x;
+        f[e] = ok[e] ? row[x[e]] : 0.f;
+      }
     }
-  }
-  {
-    const int x = 4 * n4hi + (int)threadIdx.x;  // tail of fewer than 4 keys
-    const bool ok = x < hi;
-    visit(ok, ok ? row[x] : 0.f, x);
+    unsigned int up = 0, cb = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const unsigned int bin = order_key(f[e]) >> kBinShift;
+      up += (ok[e] && bin > B) ? 1u : 0u;
+      cb += (ok[e] && bin == B) ? 1u : 0u;
+    }
+    // both counts fit 16 bits: at most 8 per thread and 8192 per block
+    const unsigned int packed = up | (cb << 16);
+    const unsigned int incl = block_scan(packed, warp_tot, &s_total);
+    const unsigned int excl = incl - packed;
+    if (threadIdx.x == 0) {
+      const unsigned int tot = s_total;
+      s_base_out = (tot & 0xFFFFu) ? atomicAdd(cnt, tot & 0xFFFFu) : 0u;
+      s_base_cand = (tot >> 16) ? atomicAdd(ncand, tot >> 16) : 0u;
+    }
+    __syncthreads();
+    unsigned int po = s_base_out + (excl & 0xFFFFu), pc = s_base_cand + (excl >> 16);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const unsigned int key = order_key(f[e]);
+      const unsigned int bin = key >> kBinShift;
+      if (ok[e] && bin > B) put(out, k, (int)po++, x[e], err, 10);
+      if (ok[e] && bin == B) {
+        if (pc < (unsigned)kCap) {
+          ck[pc] = key;
+          ci[pc] = x[e];
+        }
+        ++pc;
+      }
+    }
+    __syncthreads();  // s_base_* are rewritten by the next round
   }
 }
 
