@@ -7,7 +7,10 @@ One JSON line on rank 0.  The headline `value` is prefill tokens/s of the
 heads over a 576/512 MLA row, score tiles of 4096 query rows).  One step is
 one pass of that prefill through the three steps (indexer -> top-k per query
 block, then sparse attention).  The `decode` object reports the 128K decode
-(B=8 sequences, one query each) the same way, which adds the split-k combine.
+(B=8 sequences, one query each), which adds the split-k combine; its step is
+a few microsecond launches, so it is captured once as a CUDA graph and timed
+by replay (per-kernel times from one graph per launch group), falling back
+to eager steps if the capture fails or its selection differs.
 
 Kernel timing: each step calls the C-ABI step entry points in the order
 dsa_forward uses, with CUDA events between launches on the launching stream,
@@ -240,6 +243,21 @@ class DsaRunner:
         if ev is not None:
             ev.append(("sparse_attn", e3, e4))
 
+    def step_part(self, name):
+        """One of the step's launch groups alone (indexer, topk or sparse_attn)."""
+        d, wl, i, o = self.dsa, self.wl, self.inp, self.outs
+        qb = self.rows_per_block()
+        if name == "sparse_attn":
+            d.sparse_attn(self.shape, i["q"], i["kv"], o.idx, o.out, o.lse, self.ws)
+            return
+        for q0 in range(0, wl.T, qb):
+            cnt = min(qb, wl.T - q0)
+            if name == "indexer":
+                d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt,
+                                 self.scores)
+            else:
+                d.topk(self.shape, self.scores, q0, cnt, o.idx, self.topk_ws)
+
     def forward(self):
         self.dsa.forward(self.shape, self.inp, self.outs.out, self.outs.lse, self.outs.idx, self.ws)
 
@@ -276,6 +294,78 @@ def time_steps(runner, steps, warmup, ws):
     if st != 0:
         raise RuntimeError(f"device error {st} detail {det:#x}")
     return total_ms, per_kernel, launches
+
+
+def capture_step_graphs(runner, warmup):
+    """Decode steps are a few microsecond launches, so the bench times them by
+    CUDA-graph replay: the step is captured once, and each launch group once
+    more on its own for the per-kernel split.  No collective here.  Returns
+    ({"step", "indexer", "topk", "sparse_attn"} graphs, launches per step), or
+    None when capture or replay fails or the replayed selection differs from
+    the eager one (compared as sets per row)."""
+    d = runner.dsa
+    graphs = {}
+    try:
+        for _ in range(warmup):
+            runner.step()
+        torch.cuda.synchronize()
+        if d.device_error()[0] != 0:
+            return None
+        ref = torch.sort(runner.outs.idx, dim=-1).values
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            runner.step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        n0 = d.launch_count()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            runner.step()
+        launches = d.launch_count() - n0
+        graphs["step"] = g
+        for name in ("indexer", "topk", "sparse_attn"):
+            gp = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gp, capture_error_mode="relaxed"):
+                runner.step_part(name)
+            graphs[name] = gp
+        runner.outs.idx.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        if launches <= 0 or d.device_error()[0] != 0:
+            return None
+        if not torch.equal(torch.sort(runner.outs.idx, dim=-1).values, ref):
+            return None
+        return graphs, launches
+    except Exception:
+        return None
+
+
+def time_graphs(graphs, steps, warmup, ws):
+    """Replay timing of captured step graphs; same barriers and flushes as
+    time_steps.  Returns (total_ms, per_kernel)."""
+    flush = Flusher()
+    for _ in range(warmup):
+        graphs["step"].replay()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+
+    def timed(g):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    total_ms = sum(timed(graphs["step"]) for _ in range(steps))
+    per_kernel = {name: [timed(graphs[name]) for _ in range(steps)] for name in ("indexer", "topk", "sparse_attn")}
+    torch.cuda.synchronize()
+    barrier(ws)
+    return total_ms, per_kernel
 
 
 def kernel_report(wl, per_kernel, steps, peaks, peak_src, sustained):
@@ -398,12 +488,25 @@ def gpu_arm(args):
     dec = None
     if wl_dec is not None:
         drun = DsaRunner(wl_dec, seed_offset=rank)
-        d_total, d_kern, d_launch = time_steps(drun, args.steps, args.warmup, ws)
+        got = capture_step_graphs(drun, args.warmup)
+        # every rank takes the same path: graphs only if all ranks captured
+        use_graph = max_over_ranks(0.0 if got is not None else 1.0, ws) == 0.0
+        if use_graph:
+            timing = "cuda_graph_replay"
+            d_total, d_kern = time_graphs(got[0], args.steps, args.warmup, ws)
+            d_launch = got[1]
+        else:
+            timing = "eager"
+            d_total, d_kern, d_launch = time_steps(drun, args.steps, args.warmup, ws)
+            d_launch //= args.steps
+        if got is not None:
+            got[0].clear()
+            torch.cuda.synchronize()
         d_ms = max_over_ranks(d_total / args.steps, ws)
         d_rep = kernel_report(drun.wl, d_kern, args.steps, peaks, peak_src, sustained=False)
         d_top = max(d_rep.items(), key=lambda kv: kv[1]["ms_per_step"])
         dec = {"workload": wl_dec.name, "value": ws * wl_dec.B * wl_dec.T / (d_ms / 1e3), "unit": "tokens/s",
-               "ms_per_step": d_ms, "gpu_launches": d_launch,
+               "ms_per_step": d_ms, "gpu_launches": d_launch, "timing": timing,
                "config": {"batch": wl_dec.B, "context": wl_dec.S, "k": wl_dec.k, "H": wl_dec.H,
                           "H_I": wl_dec.H_I, "D_I": wl_dec.D_I, "d_k": wl_dec.d_k, "d_v": wl_dec.d_v},
                "roofline": {"kernel": d_top[0], "bound": d_top[1]["bound"], "achieved": d_top[1]["achieved"],
