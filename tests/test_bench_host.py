@@ -1,0 +1,58 @@
+"""Host-side arithmetic of bench.py (no GPU): the algorithmic work behind the
+roofline fractions, and the guard on the captured DRAM traffic."""
+import hashlib
+import importlib.util
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_causal_pairs_closed_forms(bench):
+    """Pair counts equal the closed forms of the causal O(L k) work.
+
+    Indexer: sum over queries of pos + 1.  Attention: sum of min(pos + 1, k).
+    """
+    from long_context_05_b200.inputs import WORKLOADS
+    wl = WORKLOADS["prefill_128k"]
+    ip, ap = bench.causal_pairs(wl)
+    L, k = wl.T, wl.k
+    assert ip == L * (L + 1) // 2 == 8_590_000_128
+    assert ap == k * (k + 1) // 2 + (L - k) * k == 266_339_328
+    dec = WORKLOADS["decode_128k_b8"]
+    ip, ap = bench.causal_pairs(dec)
+    assert ip == dec.B * dec.S and ap == dec.B * dec.k
+
+
+def test_algorithmic_flops_per_pair(bench):
+    """The roofline's work: 2 H_I D_I FLOP per indexer pair and
+    2 H (d_k + d_v) FLOP per attention pair (128K prefill: 1.407e14 and 7.42e13)."""
+    from long_context_05_b200.inputs import WORKLOADS
+    wl = WORKLOADS["prefill_128k"]
+    peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 1000.0, "hbm_gbs": 1000.0}
+    per_kernel = {"indexer": [1000.0], "topk": [1000.0], "sparse_attn": [1000.0]}  # 1 s each
+    rep = bench.kernel_report(wl, per_kernel, 1, peaks, "test", sustained=True)
+    assert rep["indexer"]["achieved"] == pytest.approx(2 * 64 * 128 * 8_590_000_128 / 1e12)
+    assert rep["sparse_attn"]["achieved"] == pytest.approx(2 * 128 * (576 + 512) * 266_339_328 / 1e12)
+    assert rep["topk"]["achieved"] == pytest.approx(4 * 8_590_000_128 / 1e9)
+
+
+def test_traffic_reported_only_for_the_captured_source(bench):
+    """roofline.traffic is the captured figure only for the captured
+    (workload, kernel) and only while the kernel source is unchanged."""
+    t = bench.ATTN_TRAFFIC
+    with open(os.path.join(ROOT, t["source"]), "rb") as f:
+        same = hashlib.sha256(f.read()).hexdigest() == t["sha256"]
+    got = bench.measured_traffic("prefill_128k", "sparse_attn")
+    assert got == (t["bytes"] if same else None)
+    assert bench.measured_traffic("prefill_8k", "sparse_attn") is None
+    assert bench.measured_traffic("prefill_128k", "indexer") is None
