@@ -127,7 +127,12 @@ DSA_API dsa_status dsa_indexer_scores(const dsa_shape* shape, const uint8_t* q_I
  * idx[b, t, 0..k) for t in [q_begin, q_begin + q_count): the indices of the
  * min(k, pos(t) + 1) largest scores, ties going to the lower index, in no
  * particular order, followed by -1 in the unused slots.  -0.0 and +0.0 count
- * as equal.  ws may be NULL (this step needs no workspace today). */
+ * as equal.  ws is optional scratch.  For few long rows (B * q_count * 2
+ * below the SM count and S >= 16384, as in decode), if ws_bytes is at least
+ * 73,744 bytes per row (ws 16-byte aligned), each row is split over 16
+ * blocks: histogram, candidate collection, then a per-row selection.
+ * Otherwise, or with ws NULL, one block handles each row.  dsa_forward
+ * reserves this scratch inside dsa_workspace_size. */
 DSA_API dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
                     int64_t ld_scores, int q_begin, int q_count, int32_t* idx,
                     void* ws, size_t ws_bytes, void* stream);
