@@ -17,14 +17,19 @@
 // sub-tiles, so each byte of k_I fetched serves 8 MMAs.  Tiles entirely
 // above the causal diagonal are skipped.
 //
-// Warp roles (448 threads, one CTA per SM, persistent over the work items):
+// Warp roles (one CTA per SM, persistent over the work items):
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..13 epilogue: three groups of four warps (one per TMEM lane
-//               quarter); group g drains sub-tiles u with u % 3 == g, so
-//               three warps per SM sub-partition hide each other's latency
-// Four TMEM accumulators of 128 columns each let the MMA run up to three
-// sub-tiles ahead of the epilogue.
+//   warps 2..   epilogue: groups of four warps (one per TMEM lane quarter);
+//               group g drains accumulator groups u with u % NGRP == g
+// Four TMEM accumulators of 128 columns each.  With 32 or more indexer heads
+// two consecutive key tiles share one accumulator group (two accumulators,
+// one commit), so every head-weight load in the epilogue serves both; two
+// epilogue groups then drain the two groups in flight (320 threads).  With
+// fewer heads each key tile has its own accumulator and three epilogue
+// groups run (448 threads), the MMA up to three sub-tiles ahead.  Items with
+// at most half of the B sub-tiles in use (decode) double-buffer B, so the
+// next item's loads overlap the current item's MMAs.
 #include "internal.h"
 #include "sm100.cuh"
 #include "tma_host.h"
