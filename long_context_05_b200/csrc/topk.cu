@@ -9,7 +9,11 @@
 // must be cache-aware).
 //
 // Keys: scores mapped to order-preserving 32-bit unsigned keys (-0.0 folded
-// onto +0.0).  Method, one block of 1024 threads per row:
+// onto +0.0).  One block of 1024 threads per row first tries a single pass:
+// a radix select over a strided sample of the row gives a lower bound on the
+// k-th key, one pass collects every key at or above it into shared memory,
+// and step 3 below selects among them.  When the bound admits fewer than k
+// keys or more than shared memory holds, the two-pass method runs:
 //   1. one pass over the row builds a 2048-bin histogram of the top 11 key
 //      bits; a block scan finds the bin B holding the k-th largest key;
 //   2. a second pass (the row is now in L2) writes every key above bin B to
