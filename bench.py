@@ -188,6 +188,18 @@ def causal_pairs(wl):
     return ip * wl.B, ap * wl.B
 
 
+def dense_rows(wl):
+    """Query rows whose visible keys all fit in k: the path keeps every one of
+    them, so it scores and selects nothing for them (dsa_forward's rule)."""
+    return max(0, min(wl.T, wl.k - (wl.S - wl.T)))
+
+
+def scored_pairs(wl):
+    """Indexer pairs the path scores: causal pairs of the rows past dense_rows."""
+    d = dense_rows(wl)
+    return wl.B * sum(wl.S - wl.T + t + 1 for t in range(d, wl.T))
+
+
 # ------------------------------------------------------------------ GPU arm
 
 class DsaRunner:
@@ -227,7 +239,15 @@ class DsaRunner:
             e.record(self.stream)
             return e
 
-        for q0 in range(0, wl.T, qb):
+        dr = dense_rows(wl)
+        if dr:
+            # rows that keep all their visible keys: the index fill only
+            e0 = mark()
+            d.topk(self.shape, self.scores, 0, dr, o.idx, self.topk_ws)
+            e1 = mark()
+            if ev is not None:
+                ev.append(("topk", e0, e1))
+        for q0 in range(dr, wl.T, qb):
             cnt = min(qb, wl.T - q0)
             e0 = mark()
             d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, self.scores)
@@ -250,7 +270,10 @@ class DsaRunner:
         if name == "sparse_attn":
             d.sparse_attn(self.shape, i["q"], i["kv"], o.idx, o.out, o.lse, self.ws)
             return
-        for q0 in range(0, wl.T, qb):
+        dr = dense_rows(wl)
+        if dr and name == "topk":
+            d.topk(self.shape, self.scores, 0, dr, o.idx, self.topk_ws)
+        for q0 in range(dr, wl.T, qb):
             cnt = min(qb, wl.T - q0)
             if name == "indexer":
                 d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt,
@@ -369,13 +392,18 @@ def time_graphs(graphs, steps, warmup, ws):
 
 
 def kernel_report(wl, per_kernel, steps, peaks, peak_src, sustained):
-    ip, ap = causal_pairs(wl)
+    _, ap = causal_pairs(wl)
+    ip = scored_pairs(wl)
     bf16 = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     kind = "sustained" if sustained else "burst"
     work = {
         # name: (algorithmic amount per step, unit, bound, peak, peak note)
-        "indexer": (2.0 * wl.H_I * wl.D_I * ip / 1e12, "TFLOP/s", "tensor", bf16 * FP8_PER_BF16,
-                    f"fp8 = {kind} bf16 x {FP8_PER_BF16:g} ({peak_src})"),
+        # decode: one query per sequence, so the indexer streams every key
+        # once (D_I FP8 bytes + a 4-byte scale) and is bound by HBM
+        "indexer": ((2.0 * wl.H_I * wl.D_I * ip / 1e12, "TFLOP/s", "tensor", bf16 * FP8_PER_BF16,
+                     f"fp8 = {kind} bf16 x {FP8_PER_BF16:g} ({peak_src})") if not wl.decode else
+                    (wl.B * wl.S * (wl.D_I + 4) / 1e9, "GB/s", "hbm", peaks["hbm_gbs"],
+                     f"hbm, k_I + k_scale bytes ({peak_src})")),
         "topk": (4.0 * ip / 1e9, "GB/s", "hbm", peaks["hbm_gbs"], f"hbm ({peak_src})"),
         "sparse_attn": ((2.0 * wl.H * (wl.d_k + wl.d_v) * ap / 1e12, "TFLOP/s", "tensor", bf16,
                          f"bf16 {kind} ({peak_src})") if not wl.decode else

@@ -22,23 +22,46 @@
  * prefill has T == S (pos = t); a decode step has T == 1 (pos = S - 1, all S
  * keys visible).
  *
+ * Positions with per-sequence lengths.  With shape->seqlens set, sequence b
+ * holds L_b = seqlens[b] keys (T <= L_b <= S) and its query t sits at
+ * pos(t) = (L_b - T) + t; keys s >= L_b are never read.  A ragged decode batch
+ * (each sequence at its own length) is T == 1 with seqlens.  S stays the row
+ * stride of the contiguous caches and the bound of every L_b.
+ *
+ * Paged caches.  With shape->page_size > 0, the key-side inputs (k_I,
+ * k_scale, kv and a separate v) are pools of num_pages * page_size token rows
+ * instead of [B, S, ...] arrays: token s of sequence b lives in row
+ *   block_table[b * pages_per_seq + s / page_size] * page_size + s % page_size.
+ * page_size must be a multiple of 16.  Pages holding no key below L_b are
+ * never read, so their block_table entries may be anything; an entry of a
+ * page that is read and lies outside [0, num_pages) is reported as
+ * DSA_ERR_DEVICE_BOUNDS and its keys read as zeros.
+ *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers to contiguous row-major arrays in
- *    the layouts stated below, owned by the caller.  The library allocates no
- *    memory on any call; scratch comes from the caller's workspace.
+ *    the layouts stated below, owned by the caller.  Scratch comes from the
+ *    caller's workspace.  The one exception is dsa_topk_static, whose scratch
+ *    is a fixed array inside this library (see its comment below).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    call only enqueues work on it and returns; nothing synchronises the host
- *    except dsa_get_device_error().
+ *    except dsa_get_device_error().  Exception: the first call of
+ *    dsa_topk_static on a device looks up its array's address (see there).
+ *  - The library caches, per device, the device addresses of its own error
+ *    word and static array.  They stay valid for the life of the CUDA
+ *    context; after cudaDeviceReset (or anything else that destroys the
+ *    primary context) reload the library before calling it again.
  *  - The current CUDA device must be the one that owns the buffers.
  *  - Argument and shape problems are reported synchronously through the
  *    return value, before anything is enqueued.  A failed launch returns
  *    DSA_ERR_CUDA.  Conditions found on the device (a bounded wait that gave
- *    up, an index out of range) never trap: they are recorded in a device
- *    error word that dsa_get_device_error() reads and clears.  No C++
+ *    up, an index or a length out of range) never trap: they are recorded in
+ *    a device error word that dsa_get_device_error() reads and clears.  No C++
  *    exception crosses this interface.
  *  - Preconditions not checked on the host: q_scale and k_scale finite and
  *    > 0 (this is what lets the kernels apply the scales after the ReLU);
- *    no NaN in the FP8 or BF16 inputs; idx entries in [-1, S) and <= pos(t).
+ *    no NaN in the FP8 or BF16 inputs; idx entries in [-1, L_b) and <= pos(t);
+ *    T <= seqlens[b] <= S (a length outside is reported on the device and
+ *    clamped into that range).
  *
  * Supported shapes: D_I in {32, 64, 128}; H_I in {4, 8, 16, 32, 64};
  * d_k in {80, 576} with d_v in {64, 512} respectively (d_v < d_k);
@@ -78,15 +101,23 @@ typedef struct {
   int mode;             /* dsa_mode; only dsa_forward looks at it            */
   int B;                /* sequences in the batch                            */
   int T;                /* query tokens per sequence                         */
-  int S;                /* keys (context tokens) per sequence                */
+  int S;                /* keys (context tokens) per sequence, at most       */
   int H_I, D_I;         /* indexer heads and head dim                        */
   int H, d_k, d_v;      /* attention heads, key dim, value dim (V = kv[:d_v])*/
   int k;                /* keys kept per query                               */
   int q_block;          /* prefill: queries per score tile (<= 0: 4096)      */
   float softmax_scale;  /* <= 0 selects 1/sqrt(d_k)                          */
+  const int32_t* seqlens;      /* device int32[B]: keys of sequence b, or NULL
+                                  (every sequence has S keys)                */
+  int page_size;               /* 0: contiguous caches; > 0: paged caches,
+                                  tokens per page (a multiple of 16)         */
+  int pages_per_seq;           /* paged: row length of block_table           */
+  int num_pages;               /* paged: pages in each cache pool            */
+  const int32_t* block_table;  /* paged: device int32[B, pages_per_seq]      */
 } dsa_shape;
 
-/* Inputs of the whole path (device pointers). */
+/* Inputs of the whole path (device pointers).  With page_size > 0 the four
+ * key-side arrays are pools of num_pages * page_size token rows. */
 typedef struct {
   const uint8_t* q_I;      /* [B, T, H_I, D_I] FP8 e4m3 indexer queries       */
   const float* q_scale;    /* [B, T, H_I]      dequant scale per query head   */
@@ -95,6 +126,8 @@ typedef struct {
   const float* k_scale;    /* [B, S]           dequant scale per key          */
   const uint16_t* q;       /* [B, T, H, d_k]   BF16 attention queries         */
   const uint16_t* kv;      /* [B, S, d_k]      BF16 cached latent+rope rows   */
+  const uint16_t* v;       /* [B, S, d_v]      BF16 values kept apart from the
+                              keys, or NULL: V = kv[..., :d_v] (MLA)          */
 } dsa_inputs;
 
 /* Library version (major * 100 + minor). */
@@ -161,21 +194,41 @@ DSA_API dsa_status dsa_topk_static(const dsa_shape* shape, const float* scores,
                            int32_t* idx, void* stream);
 
 /* Step C -- sparse MQA/MLA attention over the selected keys.
- *   q   [B, T, H, d_k] BF16;  kv [B, S, d_k] BF16 (V = kv[..., :d_v]);
+ *   q   [B, T, H, d_k] BF16;  kv [B, S, d_k] BF16 (key = the whole row);
+ *   v_or_null [B, S, d_v] BF16 values, or NULL: V = kv[..., :d_v] (MLA, the
+ *       form of the pages; a separate V is a generalisation);
  *   idx [B, T, k] int32, -1 = empty slot (skipped), duplicates counted twice;
  *   out [B, T, H, d_v] BF16 (rounded to nearest even from FP32);
  *   lse [B, T, H] FP32 natural-log sum of exp of the scaled logits, or NULL.
- * out[b,t,h] = sum_{s in idx[b,t]} softmax_s(tau q[b,t,h].kv[b,s]) kv[b,s,:d_v].
- * A row with no valid index gives out = 0 and lse = -inf.
+ * out[b,t,h] = sum_{s in idx[b,t]} softmax_s(tau q[b,t,h].kv[b,s]) V[b,s].
+ * A row with no valid index gives out = 0 and lse = -inf.  An index outside
+ * [0, L_b) is reported as DSA_ERR_DEVICE_BOUNDS and skipped.
  * ws: dsa_workspace_size(shape) bytes (decode splits the keys and merges the
  * partial results there); may be NULL in prefill mode. */
 DSA_API dsa_status dsa_sparse_attn(const dsa_shape* shape, const uint16_t* q,
-                           const uint16_t* kv, const int32_t* idx,
-                           uint16_t* out, float* lse, void* ws,
-                           size_t ws_bytes, void* stream);
+                           const uint16_t* kv, const uint16_t* v_or_null,
+                           const int32_t* idx, uint16_t* out, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Dense causal attention of every query over all its visible keys
+ * s <= pos(t), with no indexer and no selection: the "MHA with a mask" form
+ * in which short prefills run (tenelement.pl, "DeepSeek V3.2-Exp Cuts
+ * Long-Context Costs ...", section "Efektywnosc Kosztowa").  When k covers
+ * every visible key this is exactly what the sparse path computes, and
+ * dsa_forward uses it by itself for those rows.  Arguments as for
+ * dsa_sparse_attn, without idx; ws: dsa_workspace_size(shape) bytes in
+ * decode mode (the keys of a long row are split and merged there), may be
+ * NULL in prefill mode. */
+DSA_API dsa_status dsa_dense_attn(const dsa_shape* shape, const uint16_t* q,
+                          const uint16_t* kv, const uint16_t* v_or_null,
+                          uint16_t* out, float* lse, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /* The whole path, A -> B -> C, in `shape->mode`.  Prefill scores the queries
  * in blocks of q_block rows so the T x S score matrix never exists in full.
+ * Rows whose every visible key fits in k (pos(t) + 1 <= k for any length
+ * up to S) skip steps A and B: their selection is all visible keys, written
+ * to idx_out as 0..pos(t), and step C runs on them densely.
  * idx_out: [B, T, k] int32 receives the selection (required).
  * ws: at least dsa_workspace_size(shape) bytes. */
 DSA_API dsa_status dsa_forward(const dsa_shape* shape, const dsa_inputs* in,
@@ -189,6 +242,55 @@ DSA_API dsa_status dsa_prefill(const dsa_shape* shape, const dsa_inputs* in,
 DSA_API dsa_status dsa_decode(const dsa_shape* shape, const dsa_inputs* in,
                       uint16_t* out, float* lse, int32_t* idx_out, void* ws,
                       size_t ws_bytes, void* stream);
+
+/* ---- One sequence's keys over several devices (key-split decode) ----------
+ * The pages run DSA on one device; these three calls are the exchange steps
+ * that let one long sequence's keys live on P devices (an addition of this
+ * library, resting on arithmetic, not on a passage of the pages: exact top-k
+ * decomposes over disjoint key ranges -- the whole row's winners are winners
+ * of their own range under the same order -- and exact softmax attention
+ * decomposes through the log-sum-exp).  Part r holds keys
+ * [part_begin_r, part_begin_r + S_r) and runs dsa_indexer_scores and dsa_topk
+ * on a shape with S = S_r; then
+ *   1. dsa_topk_candidates packs its selection as (score, global index);
+ *   2. the caller all-gathers the P candidate lists (NCCL, P x B*T x k pairs);
+ *   3. dsa_topk_merge gives the global top-k and this part's share of it as
+ *      local indices, which dsa_sparse_attn (shape with S = S_r) consumes;
+ *   4. the caller all-gathers the P (out, lse) pairs;
+ *   5. dsa_attn_combine merges them.
+ * Rows are every query row of the shape (B * T, decode: B). */
+
+/* (score, global index) of each selected key: reads idx [B, T, k] (local
+ * indices, -1 = empty) and the score rows [B*T, ld_scores] they index
+ * (rows as dsa_indexer_scores writes them for q_begin = 0, q_count = T);
+ * writes cand_scores [B*T, k] FP32 and cand_idx [B*T, k] int32 =
+ * part_begin + local index (-inf and -1 for empty slots).  An index >= S is
+ * reported as DSA_ERR_DEVICE_BOUNDS and written as empty. */
+DSA_API dsa_status dsa_topk_candidates(const dsa_shape* shape, const float* scores,
+                               int64_t ld_scores, const int32_t* idx,
+                               int32_t part_begin, float* cand_scores,
+                               int32_t* cand_idx, void* stream);
+
+/* Global top-k of nparts candidate lists: cand_scores / cand_idx
+ * [nparts, B*T, k] (part-major, as an all-gather stacks them).  Writes
+ * idx [B*T, k]: the k best candidates by (score descending, global index
+ * ascending), in no particular order, -1 after the last; and, if idx_local is
+ * not NULL, idx_local [B*T, k]: the same selection as indices local to the
+ * key range [local_begin, local_begin + local_count), -1 outside it.
+ * nparts * k must not exceed 8192 (DSA_ERR_UNSUPPORTED; merge in rounds). */
+DSA_API dsa_status dsa_topk_merge(const dsa_shape* shape, int nparts,
+                          const float* cand_scores, const int32_t* cand_idx,
+                          int32_t* idx, int32_t local_begin, int32_t local_count,
+                          int32_t* idx_local, void* stream);
+
+/* Merge of attention results over disjoint key subsets: o_parts
+ * [nparts, B, T, H, d_v] BF16 and lse_parts [nparts, B, T, H] FP32 (natural
+ * log, -inf = no key) as dsa_sparse_attn writes them, stacked part-major.
+ *   out = sum_r e^(lse_r - M) o_r / sum_r e^(lse_r - M),  M = max_r lse_r,
+ *   lse = M + ln sum_r e^(lse_r - M)   (lse may be NULL). */
+DSA_API dsa_status dsa_attn_combine(const dsa_shape* shape, int nparts,
+                            const uint16_t* o_parts, const float* lse_parts,
+                            uint16_t* out, float* lse, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_BOUNDS

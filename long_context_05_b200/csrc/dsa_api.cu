@@ -83,7 +83,35 @@ dsa_status check_shape(const dsa_shape* s) {
   if (s->H > 128 || s->H % 8 != 0) return DSA_ERR_UNSUPPORTED;
   if (s->k > 2048) return DSA_ERR_UNSUPPORTED;
   if ((long long)s->S >= (1LL << 31) / 8) return DSA_ERR_UNSUPPORTED;
+  if (s->page_size < 0) return DSA_ERR_INVALID_ARG;
+  if (s->page_size > 0) {
+    if (s->page_size % 16 != 0) return DSA_ERR_UNSUPPORTED;
+    if (s->block_table == nullptr || s->num_pages <= 0 ||
+        (long long)s->pages_per_seq * s->page_size < (long long)s->S)
+      return DSA_ERR_INVALID_ARG;
+    if ((long long)s->num_pages * s->page_size >= (1LL << 31) / 8) return DSA_ERR_UNSUPPORTED;
+  }
   return DSA_OK;
+}
+
+// Where each sequence's keys are (lengths, paged or contiguous caches).
+KvMap kv_map(const dsa_shape* s) {
+  KvMap m;
+  m.seqlens = s->seqlens;
+  m.block_table = s->page_size > 0 ? s->block_table : nullptr;
+  m.S = s->S;
+  m.T = s->T;
+  m.page_size = s->page_size > 0 ? s->page_size : 0;
+  m.pages_per_seq = s->page_size > 0 ? s->pages_per_seq : 0;
+  m.num_pages = s->page_size > 0 ? s->num_pages : 0;
+  return m;
+}
+
+// Query rows t < dense_rows see at most k keys for every length up to S
+// (pos(t) + 1 <= S - T + t + 1 <= k): their selection is all visible keys.
+int dense_rows_of(const dsa_shape* s) {
+  const long long d = (long long)s->k - ((long long)s->S - s->T);
+  return d <= 0 ? 0 : (d >= s->T ? s->T : (int)d);
 }
 
 int q_block_of(const dsa_shape* s) {
@@ -104,7 +132,7 @@ struct WsLayout {
   size_t part_off, part_bytes;
   size_t topk_off, topk_bytes;
   size_t total;
-  int nsplit;
+  int nsplit, nsplit_dense;
   int q_rows;
 };
 
@@ -114,8 +142,18 @@ WsLayout ws_layout(const dsa_shape* s, int num_sms) {
   L.scores_off = 0;
   L.scores_bytes = round_up((size_t)s->B * L.q_rows * scores_ld(s) * sizeof(float), 256);
   L.nsplit = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->d_v, s->k, num_sms) : 1;
+  // dense attention (dsa_dense_attn) splits a decode row's S keys instead
+  L.nsplit_dense = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->d_v, s->S, num_sms) : 1;
   L.part_off = L.scores_off + L.scores_bytes;
-  L.part_bytes = round_up(attn_partial_floats(s->B * s->T, s->H, s->d_v, L.nsplit) * sizeof(float), 256);
+  size_t pb = attn_partial_floats(s->B * s->T, s->H, s->d_v, L.nsplit) * sizeof(float);
+  const size_t pb_dense = attn_partial_floats(s->B * s->T, s->H, s->d_v, L.nsplit_dense) * sizeof(float);
+  // the decode kernel's FP16 partials (MLA rows with the selection)
+  const size_t pb_dec = s->mode == DSA_DECODE && s->d_k == 576 && s->d_v == 512
+                            ? attn_decode_partial_bytes(s->B * s->T, s->H, attn_decode_nsplit(s->k))
+                            : 0;
+  if (pb_dense > pb) pb = pb_dense;
+  if (pb_dec > pb) pb = pb_dec;
+  L.part_bytes = round_up(pb, 256);
   L.topk_off = L.part_off + L.part_bytes;
   const int topk_rows = s->B * L.q_rows;
   L.topk_bytes = topk_uses_workspace(topk_rows, s->S, num_sms) ? round_up(topk_workspace_bytes(topk_rows), 256) : 0;
@@ -129,6 +167,7 @@ dsa_status run_indexer(const LaunchCtx& c, const dsa_shape* s, const uint8_t* q_
                        const float* w, const uint8_t* k_I, const float* k_scale, int q_begin, int q_count,
                        float* scores, int64_t ld) {
   IndexerArgs a;
+  a.kv = kv_map(s);
   a.q_I = q_I; a.q_scale = q_scale; a.w = w; a.k_I = k_I; a.k_scale = k_scale;
   a.scores = scores; a.ld = ld;
   a.B = s->B; a.T = s->T; a.S = s->S; a.H_I = s->H_I; a.D_I = s->D_I;
@@ -139,19 +178,27 @@ dsa_status run_indexer(const LaunchCtx& c, const dsa_shape* s, const uint8_t* q_
 dsa_status run_topk(const LaunchCtx& c, const dsa_shape* s, const float* scores, int64_t ld, int q_begin,
                     int q_count, int32_t* idx, void* ws, size_t ws_bytes) {
   TopkArgs a;
+  a.kv = kv_map(s);
   a.scores = scores; a.ld = ld; a.idx = idx;
   a.B = s->B; a.T = s->T; a.S = s->S; a.k = s->k;
   a.q_begin = q_begin; a.q_count = q_count;
   return from_cuda(launch_topk(c, a, ws, ws_bytes));
 }
 
+// idx null: dense causal attention of every row; otherwise rows t <
+// dense_rows read keys 0..pos(t) and the rest read idx.
 dsa_status run_attn(const LaunchCtx& c, const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
-                    const int32_t* idx, uint16_t* out, float* lse, float* part, int nsplit) {
+                    const uint16_t* v, const int32_t* idx, int dense_rows, uint16_t* out, float* lse, float* part,
+                    int nsplit) {
   AttnArgs a;
-  a.q = q; a.kv = kv; a.idx = idx; a.out = out; a.lse = lse; a.part = part;
+  a.map = kv_map(s);
+  a.q = q; a.kv = kv; a.v = v; a.idx = idx; a.dense_rows = dense_rows;
+  a.out = out; a.lse = lse; a.part = part;
   a.B = s->B; a.T = s->T; a.S = s->S; a.H = s->H; a.d_k = s->d_k; a.d_v = s->d_v; a.k = s->k;
   a.nsplit = nsplit;
   a.tau = tau_of(s);
+  a.decode = s->mode == DSA_DECODE;
+  if (a.decode && attn_decode_supported(a)) return from_cuda(launch_sparse_attn_decode(c, a, part));
   return from_cuda(launch_sparse_attn(c, a));
 }
 
@@ -171,7 +218,7 @@ using namespace dsa;
 
 extern "C" {
 
-int dsa_version(void) { return 100; }
+int dsa_version(void) { return 200; }
 
 const char* dsa_status_string(dsa_status st) {
   switch (st) {
@@ -227,20 +274,38 @@ dsa_status dsa_topk(const dsa_shape* s, const float* scores, int64_t ld_scores, 
   return run_topk(c, s, scores, ld_scores, q_begin, q_count, idx, ws, ws_bytes);
 }
 
-dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv, const int32_t* idx,
-                           uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv, const uint16_t* v,
+                           const int32_t* idx, uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
   dsa_status st = check_shape(s);
   if (st != DSA_OK) return st;
-  if (!q || !kv || !idx || !out || !aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (!q || !kv || !idx || !out || !aligned16(q) || !aligned16(kv) || !aligned16(out) || (v && !aligned16(v)))
+    return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
   WsLayout L = ws_layout(s, c.num_sms);
   float* part = nullptr;
-  if (L.part_bytes > 0) {
+  if (L.nsplit > 1 || (s->mode == DSA_DECODE && attn_decode_nsplit(s->k) > 1)) {
     if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
     part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.part_off);
   }
-  return run_attn(c, s, q, kv, idx, out, lse, part, L.nsplit);
+  return run_attn(c, s, q, kv, v, idx, 0, out, lse, part, L.nsplit);
+}
+
+dsa_status dsa_dense_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv, const uint16_t* v,
+                          uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  dsa_status st = check_shape(s);
+  if (st != DSA_OK) return st;
+  if (!q || !kv || !out || !aligned16(q) || !aligned16(kv) || !aligned16(out) || (v && !aligned16(v)))
+    return DSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
+  WsLayout L = ws_layout(s, c.num_sms);
+  float* part = nullptr;
+  if (L.nsplit_dense > 1) {
+    if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.part_off);
+  }
+  return run_attn(c, s, q, kv, v, nullptr, 0, out, lse, part, L.nsplit_dense);
 }
 
 dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, float* lse, int32_t* idx_out,
@@ -249,7 +314,8 @@ dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, 
   if (st != DSA_OK) return st;
   if (in == nullptr || out == nullptr || idx_out == nullptr) return DSA_ERR_INVALID_ARG;
   if (!indexer_ptrs_ok(in->q_I, in->q_scale, in->w, in->k_I, in->k_scale)) return DSA_ERR_INVALID_ARG;
-  if (!in->q || !in->kv || !aligned16(in->q) || !aligned16(in->kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (!in->q || !in->kv || !aligned16(in->q) || !aligned16(in->kv) || !aligned16(out) || (in->v && !aligned16(in->v)))
+    return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
   WsLayout L = ws_layout(s, c.num_sms);
@@ -257,7 +323,12 @@ dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, 
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + L.scores_off);
   float* part = L.part_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) + L.part_off) : nullptr;
   const int64_t ld = scores_ld(s);
-  for (int q0 = 0; q0 < s->T; q0 += L.q_rows) {
+  // rows whose visible keys all fit in k: no scores, the selection is 0..pos
+  const int d_rows = dense_rows_of(s);
+  if (d_rows > 0 &&
+      (st = run_topk(c, s, scores, ld, 0, d_rows, idx_out, nullptr, 0)) != DSA_OK)
+    return st;
+  for (int q0 = d_rows; q0 < s->T; q0 += L.q_rows) {
     const int cnt = (s->T - q0) < L.q_rows ? (s->T - q0) : L.q_rows;
     if ((st = run_indexer(c, s, in->q_I, in->q_scale, in->w, in->k_I, in->k_scale, q0, cnt, scores, ld)) != DSA_OK)
       return st;
@@ -265,7 +336,7 @@ dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, 
                        L.topk_bytes ? static_cast<char*>(ws) + L.topk_off : nullptr, L.topk_bytes)) != DSA_OK)
       return st;
   }
-  return run_attn(c, s, in->q, in->kv, idx_out, out, lse, part, L.nsplit);
+  return run_attn(c, s, in->q, in->kv, in->v, idx_out, d_rows, out, lse, part, L.nsplit);
 }
 
 dsa_status dsa_prefill(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, float* lse, int32_t* idx_out,

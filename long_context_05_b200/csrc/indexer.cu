@@ -59,6 +59,9 @@ struct EpiCfg {
 };
 
 struct IdxParams {
+  KvMap kv;            // per-sequence lengths, paged or contiguous key cache
+  long long pool_rows; // rows of the k_I / k_scale pools
+  int box_rows;        // key rows per TMA load (a key tile takes kBM / box_rows)
   const float* w;
   const float* q_scale;
   const float* k_scale;
@@ -93,6 +96,8 @@ struct Layout {
 // key chunk); CTA `cta` takes every item whose flat index is cta mod grid.
 struct Item {
   int b, t0, tend, c, ntiles;
+  int L;    // keys of sequence b
+  int off;  // L - T: pos(t) = off + t
 };
 
 template <int HI, class F>
@@ -107,9 +112,11 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
     const int g = gid - b * p.groups_per_seq;
     Item it;
     it.b = b;
+    it.L = p.kv.len(b, p.err, ERR_SITE_INDEXER);
+    it.off = it.L - p.T;
     it.t0 = p.q_begin + g * per_group;
     it.tend = min(it.t0 + per_group, q_end);
-    const int pos_last = p.S - p.T + it.tend - 1;
+    const int pos_last = it.off + it.tend - 1;
     it.ntiles = pos_last / kBM + 1;
     const int nch = (it.ntiles + p.kc - 1) / p.kc;
     int c0 = (int)(((long long)cta - flat) % grid);
@@ -135,8 +142,8 @@ __device__ __forceinline__ int item_nsub(const IdxParams& p, const Item& it) {
 template <int HI>
 __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, int kt, int nsub) {
   constexpr int QPS = kNSub / HI;
-  // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM - (S - T)
-  const int x = kt * kBM - (p.S - p.T) - it.t0 + QPS;
+  // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM - off
+  const int x = kt * kBM - it.off - it.t0 + QPS;
   const int j = x > 0 ? x / QPS - 1 : 0;
   return j < 0 ? 0 : (j < nsub - 1 ? j : nsub - 1);
 }
@@ -234,7 +241,18 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
             fail(2); ok = false; return false;
           }
           mbar_arrive_expect_tx(&a_full[st], L::kABytes);
-          tma_load_2d(sA + st * L::kABytes, &tm_k, &a_full[st], 0, it.b * p.S + kt * kBM);
+          // the tile's keys in runs of box_rows cache rows (a whole tile when
+          // the cache is contiguous); a run at or past L_b, or on an unmapped
+          // page, reads the fill value from past the end of the pool
+          for (int r0 = 0; r0 < kBM; r0 += p.box_rows) {
+            const int s = kt * kBM + r0;
+            long long y = s < it.L ? p.kv.row(it.b, s) : -1;
+            if (y < 0) {
+              if (s < it.L) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (2u << 8));
+              y = p.pool_rows;
+            }
+            tma_load_2d(sA + st * L::kABytes + r0 * DI, &tm_k, &a_full[st], 0, (int)y);
+          }
           issued[st] = true;
           last_phase[st] = (a_cnt / kStages) & 1;
         }
@@ -349,7 +367,8 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
         for (int g = 0; g < E::G; ++g) {
           sg[g] = (kt + g) * kBM + r;
           // 1/2: the head sum below accumulates 2 ReLU(x)
-          ksg[g] = (g < ng && sg[g] < p.S) ? 0.5f * p.k_scale[(size_t)it.b * p.S + sg[g]] : 0.f;
+          const long long kr = (g < ng && sg[g] < it.L) ? p.kv.row(it.b, sg[g]) : -1;
+          ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
         }
         const int jlo = first_active<HI>(p, it, kt, nsub);
         const uint32_t u0 = u;
@@ -428,7 +447,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
 #pragma unroll
               for (int i = 0; i < NP; ++i) a += part[g][q][i].x + part[g][q][i].y;
               const int t = it.t0 + j * QPS + q;
-              if (t < it.tend && s <= p.S - p.T + t) {
+              if (t < it.tend && s <= it.off + t) {
                 // self-check: the score slot lies inside this launch's tile
                 const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
                 if (ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld)
@@ -460,11 +479,21 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   const CUtensorMapSwizzle sw = DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : DI == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                            : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (!make_tmap_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.k_I, (uint64_t)a.B * a.S, DI, DI, kBM, DI, sw))
+  // key rows per TMA load: a whole tile, or the largest power of two that
+  // divides the page size (every load then stays inside one page)
+  int box_rows = kBM;
+  if (a.kv.page_size > 0)
+    while (a.kv.page_size % box_rows != 0) box_rows >>= 1;
+  const long long pool_rows = a.kv.pool_rows(a.B);
+  if (box_rows < 16 || pool_rows <= 0 || pool_rows >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.k_I, (uint64_t)pool_rows, DI, DI, box_rows, DI, sw))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_I, (uint64_t)a.B * a.T * HI, DI, DI, kNSub, DI, sw))
     return cudaErrorInvalidValue;
   IdxParams p;
+  p.kv = a.kv;
+  p.pool_rows = pool_rows;
+  p.box_rows = box_rows;
   p.w = a.w;
   p.q_scale = a.q_scale;
   p.k_scale = a.k_scale;

@@ -30,6 +30,44 @@ __device__ __forceinline__ void report_error(DevErr* e, unsigned int code, unsig
 }
 #endif
 
+// Where the keys of each sequence are: per-sequence lengths and the
+// (optionally paged) layout of the key-side caches.
+struct KvMap {
+  const int32_t* seqlens;      // device int32[B] or null (every sequence has S keys)
+  const int32_t* block_table;  // device int32[B, pages_per_seq] (paged only)
+  int S;                       // keys per sequence at most; row stride when contiguous
+  int T;                       // queries per sequence (a length below T is clamped up)
+  int page_size;               // 0: contiguous [B, S, ...] caches
+  int pages_per_seq, num_pages;
+
+#ifdef __CUDACC__
+  // Keys of sequence b, L_b.  A length outside [T, S] is reported once per
+  // calling thread and clamped into that range.
+  __device__ __forceinline__ int len(int b, DevErr* err, unsigned site) const {
+    if (seqlens == nullptr) return S;
+    const int L = seqlens[b];
+    if (L < T || L > S) {
+      report_error(err, DSA_ERR_DEVICE_BOUNDS, site | (0xB0u << 8));
+      return L < T ? T : S;
+    }
+    return L;
+  }
+  // Cache row of token s of sequence b, or -1 when its page is not mapped.
+  __device__ __forceinline__ long long row(int b, int s) const {
+    if (page_size == 0) return (long long)b * S + s;
+    const int pg = s / page_size;
+    if (pg < 0 || pg >= pages_per_seq) return -1;
+    const int e = block_table[(size_t)b * pages_per_seq + pg];
+    if (e < 0 || e >= num_pages) return -1;
+    return (long long)e * page_size + (s - pg * page_size);
+  }
+#endif
+  // rows in each cache pool (contiguous: B * S)
+  long long pool_rows(int B) const {
+    return page_size == 0 ? (long long)B * S : (long long)num_pages * page_size;
+  }
+};
+
 // Everything a launcher needs besides its own arguments.
 struct LaunchCtx {
   cudaStream_t stream;
@@ -40,6 +78,7 @@ struct LaunchCtx {
 };
 
 struct IndexerArgs {
+  KvMap kv;
   const uint8_t* q_I;
   const float* q_scale;
   const float* w;
@@ -52,6 +91,7 @@ struct IndexerArgs {
 };
 
 struct TopkArgs {
+  KvMap kv;                 // only the lengths are used
   const float* scores;
   int64_t ld;
   int32_t* idx;
@@ -60,15 +100,19 @@ struct TopkArgs {
 };
 
 struct AttnArgs {
+  KvMap map;
   const uint16_t* q;
   const uint16_t* kv;
-  const int32_t* idx;
+  const uint16_t* v;   // separate values [.., d_v] or null (V = kv[.., :d_v])
+  const int32_t* idx;  // null: dense causal attention over every visible key
+  int dense_rows;      // query rows t < dense_rows take all visible keys (idx not read)
   uint16_t* out;
   float* lse;
   float* part;         // split partials [rows, nsplit, H, d_v + 2] or null
   int B, T, S, H, d_k, d_v, k;
   int nsplit;          // key splits per query row (1 = write out directly)
   float tau;
+  bool decode;         // decode mode: the split-k memory-bound kernel where it applies
 };
 
 // counts every kernel launch (dsa_launch_count)
@@ -84,6 +128,11 @@ constexpr int kTopkHistBins = 2048;
 bool topk_uses_workspace(int rows, int S, int num_sms);
 cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a);
 
+// key-split rows (one sequence's keys over several parts; split.cu, topk.cu)
+cudaError_t launch_topk_merge(const LaunchCtx& c, const float* cand_scores, const int32_t* cand_idx, int rows,
+                              int nparts, int k, int32_t* idx, int local_begin, int local_count, int32_t* idx_local);
+int topk_merge_max_candidates();
+
 cudaError_t launch_wait_timeout_probe(const LaunchCtx& c);
 
 // shape validation and launch context of the public entry points (dsa_api.cu)
@@ -93,5 +142,12 @@ dsa_status api_make_ctx(void* stream, LaunchCtx* c);
 // split-k partial buffer size (floats) for a decode attention launch
 size_t attn_partial_floats(int rows, int H, int d_v, int nsplit);
 int attn_choose_nsplit(int rows, int H, int d_v, int k, int num_sms);
+
+// the decode kernel (sparse_attn_decode.cu): MLA rows (d_k 576, d_v 512, V in
+// the key row), splits of 128 selected slots, FP16 partials + FP32 LSE
+bool attn_decode_supported(const AttnArgs& a);
+int attn_decode_nsplit(int k);
+size_t attn_decode_partial_bytes(int rows, int H, int nsplit);
+cudaError_t launch_sparse_attn_decode(const LaunchCtx& c, const AttnArgs& a, void* part);
 
 }  // namespace dsa

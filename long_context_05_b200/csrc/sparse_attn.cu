@@ -54,7 +54,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kSlotKeys = 32;   // keys per gather slot
-constexpr int kSlots = 4;       // gather ring slots
 constexpr int kN = 2 * kSlotKeys;  // keys per chunk = N of Q K^T (two adjacent slots)
 constexpr int kSBuf = 2;        // S/P buffers in TMEM
 // Warps: 0 MMA, 1-3 gather the even slot of every chunk, 4-11 softmax (two
@@ -69,12 +68,20 @@ constexpr int kThreads = 32 * (kFirstGatherB + kGatherPerSlot);
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
-template <int DK, int DV>
+// SEPV: values come from their own array (not the first DV columns of the
+// key row); each slot then also holds this CTA's value atoms, and the ring
+// shrinks to one chunk of two slots to make room.
+template <int DK, int DV, bool SEPV = false>
 struct Cfg {
   static constexpr int KSTEPS = DK / 16;             // 16-wide MMA K steps over the key dim
-  static constexpr int NATOM = (DK + 63) / 64;       // 64-column (128-byte) atoms of a row
+  static constexpr int NATOM = (DK + 63) / 64;       // 64-column (128-byte) atoms of a key row
   static constexpr int NHALF = DV >= 128 ? 2 : 1;    // value columns split over CTAs
   static constexpr int DVH = DV / NHALF;
+  static constexpr int NVATOM = (DVH + 63) / 64;     // value atoms of this CTA's half
+  static constexpr int ATOMS = NATOM + (SEPV ? NVATOM : 0);  // atoms gathered per key
+  static constexpr int SLOTS = SEPV ? 2 : 4;         // gather ring slots
+  static constexpr int NCH = SLOTS / 2;              // chunks held by the ring
+  static constexpr int VATOM0 = SEPV ? NATOM : 0;    // first atom read as V (plus half * NVATOM when !SEPV)
   static constexpr uint32_t OCOL = 0;
   static constexpr uint32_t SCOL = (DVH + 31) / 32 * 32;
   static constexpr uint32_t QCOL = SCOL + kSBuf * kN;
@@ -86,16 +93,16 @@ struct Cfg {
   static constexpr int QS_ATOMS = (DK - QT_DIMS) / 64;   // Q atoms in shared memory
   static constexpr int Q_ATOM = 128 * 128;               // 128 head rows x 128 bytes
   static constexpr int SLOT_ATOM = kSlotKeys * 128;
-  static constexpr int ATOM_STRIDE = kSlots * SLOT_ATOM;
-  static constexpr int RING = NATOM * ATOM_STRIDE;
+  static constexpr int ATOM_STRIDE = SLOTS * SLOT_ATOM;
+  static constexpr int RING = ATOMS * ATOM_STRIDE;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + QS_ATOMS * Q_ATOM;
   static constexpr int OFF_MASK = OFF_KV + RING;
   // partial row maxima exchanged by the two softmax warps of a lane quarter,
   // one set per S buffer: [kSBuf][2 sides][128 rows]
-  static constexpr int OFF_XM = OFF_MASK + kSlots * 4;
+  static constexpr int OFF_XM = OFF_MASK + SLOTS * 4;
   static constexpr int OFF_BAR = OFF_XM + kSBuf * 2 * 128 * 4;
-  static constexpr int NBARS = 2 + 2 * kSlots + 3 * kSBuf + 1 + kSBuf * 4 + 4;
+  static constexpr int NBARS = 2 + 2 * SLOTS + 3 * kSBuf + 1 + kSBuf * 4 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   // the dynamic shared memory base is checked for 1024-byte alignment at run
@@ -108,9 +115,13 @@ struct Cfg {
 };
 
 struct AttnParams {
+  KvMap map;        // per-sequence lengths, paged or contiguous caches
   const uint16_t* q;
   const uint16_t* kv;
-  const int32_t* idx;
+  const uint16_t* v;    // separate values (SEPV kernels only)
+  const int32_t* idx;   // null: every row dense
+  int dense_rows;       // rows with t < dense_rows take keys 0..pos(t), idx unread
+  int kslots;           // slots per row (k; the longest visible run when dense)
   uint16_t* out;
   float* lse;
   float* part_o;    // [rows, nsplit, H, d_v] (split mode)
@@ -123,23 +134,13 @@ struct AttnParams {
   DevErr* err;
 };
 
-// 2^x with the hardware approximation (flushes subnormal results to zero)
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 
-template <int DK, int DV>
+template <int DK, int DV, bool SEPV>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
-  using C = Cfg<DK, DV>;
+  using C = Cfg<DK, DV, SEPV>;
+  constexpr int kSlots = C::SLOTS;
   extern __shared__ uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {
     // self-check: the layouts below need a 1024-byte aligned base
@@ -171,10 +172,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row = rest / p.nsplit;  // b * T + t
   const int split = rest - row * p.nsplit;
   const int b = row / p.T;
+  const int t = row - b * p.T;
   const int slot0 = split * p.kc;
-  const int slot1 = min(p.k, slot0 + p.kc);
   // self-check: a CTA outside the launch's rows does no work
   const bool row_ok = row >= 0 && row < p.rows && split >= 0 && split < p.nsplit && slot0 >= 0;
+  const int Lb = row_ok ? p.map.len(b, p.err, ERR_SITE_ATTN) : 0;
+  const int pos = Lb - p.T + t;                 // this query's position
+  const bool dense = p.idx == nullptr || t < p.dense_rows;
+  // dense rows read keys 0..pos in slot order (slot i holds key i)
+  const int slot1 = min(dense ? pos + 1 : p.kslots, min(p.kslots, slot0 + p.kc));
   const int nchunks = row_ok && slot1 > slot0 ? (slot1 - slot0 + kN - 1) / kN : 0;
 
   if (threadIdx.x == 0) {
@@ -229,44 +235,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       q_issued = true;
     }
     const int c16 = lane & 7, rg = lane >> 3;  // 16-byte column chunk, row group
-    const int32_t* irow = p.idx + (size_t)row * p.k;
-    const uint16_t* kvb = p.kv + (size_t)b * p.S * DK;
+    const int32_t* irow = dense ? nullptr : p.idx + (size_t)row * p.k;
     // indices of this half of chunk j, loaded one chunk ahead
     int ivn[kSlotKeys / 4];
     auto load_idx = [&](int j) {
 #pragma unroll
       for (int m = 0; m < kSlotKeys / 4; ++m) {
         const int slot = slot0 + j * kN + h * kSlotKeys + rg + 4 * m;
-        ivn[m] = (j < nchunks && slot < slot1) ? irow[slot] : -1;
+        ivn[m] = (j < nchunks && slot < slot1) ? (dense ? slot : irow[slot]) : -1;
       }
     };
     load_idx(0);
     for (int j = 0; j < nchunks; ++j) {
-      const int st = 2 * (j % 2) + h;          // ring slot of this half of chunk j
+      const int st = 2 * (j % C::NCH) + h;     // ring slot of this half of chunk j
       int iv[kSlotKeys / 4];
 #pragma unroll
       for (int m = 0; m < kSlotKeys / 4; ++m) iv[m] = ivn[m];
-      if (j >= 2 && !wwait(&kv_empty[st], (uint32_t)((j / 2) - 1) & 1)) { fail(1); break; }
+      if (j >= C::NCH && !wwait(&kv_empty[st], (uint32_t)((j / C::NCH) - 1) & 1)) { fail(1); break; }
       uint8_t* slotp = sKV + st * C::SLOT_ATOM;
       uint32_t mask = 0;
 #pragma unroll
       for (int m = 0; m < kSlotKeys / 4; ++m) {
         const int r = rg + 4 * m;
         int v = iv[m];
-        if (v >= p.S) {
+        if (v >= Lb) {
           if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
+          v = -1;
+        }
+        long long cr = v >= 0 ? p.map.row(b, v) : -1;   // cache row of key v
+        if (v >= 0 && cr < 0) {
+          if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
           v = -1;
         }
         const bool valid = v >= 0;
         // lanes 0, 8, 16, 24 hold rows 4m .. 4m+3
         const uint32_t bal = __ballot_sync(0xffffffffu, valid);
         mask |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u)) << (4 * m);
-        const uint16_t* src = kvb + (size_t)(valid ? v : 0) * DK;
+        // an empty or invalid slot is zero-filled, so that no stale or
+        // non-finite shared memory meets its zero probability in P V
+        const uint16_t* src = p.kv + (size_t)(valid ? cr : 0) * DK;
 #pragma unroll
-        for (int a0 = 0; a0 < C::NATOM; a0 += kGatherPerSlot) {
+        for (int a0 = 0; a0 < C::ATOMS; a0 += kGatherPerSlot) {
           const int a = a0 + g;
-          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2)
-            cp_async16(slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
+          uint8_t* dst = slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4);
+          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2) {
+            if (valid) cp_async16(dst, src + a * 64 + c16 * 8);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          } else if (SEPV && a >= C::NATOM && a < C::ATOMS) {
+            // value atom: columns half * DVH + (a - NATOM) * 64 .. of the value row
+            const int vc = (a - C::NATOM) * 64 + c16 * 8;
+            if (vc < C::DVH) {
+              if (valid) cp_async16(dst, p.v + (size_t)cr * DV + half * C::DVH + vc);
+              else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
         }
       }
       if (g == 0 && lane == 0) sMask[st] = mask;
@@ -288,8 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the start-address field (no carry: shared addresses are < 256 KB)
       const uint64_t kdesc0 = make_sdesc(smem_u32(sKV), 16, 1024, kSwizzle128);
       const uint64_t qdesc0 = make_sdesc(smem_u32(sQ), 16, 1024, kSwizzle128);
-      const uint64_t vdesc0 =
-          make_sdesc(smem_u32(sKV) + (uint32_t)(half * C::DVH / 64) * C::ATOM_STRIDE, C::ATOM_STRIDE, 1024, kSwizzle128);
+      const uint64_t vdesc0 = make_sdesc(
+          smem_u32(sKV) + (uint32_t)(SEPV ? C::VATOM0 : half * C::DVH / 64) * C::ATOM_STRIDE, C::ATOM_STRIDE, 1024,
+          kSwizzle128);
       bool ok = nchunks == 0 || ((C::QS_ATOMS == 0 || mbar_wait(q_full, 0, p.wait_ns, ab)) &&
                                  mbar_wait(q_ready, 0, p.wait_ns, ab));
       if (!ok) fail(3);
@@ -608,13 +631,17 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, 
     lse[(size_t)row * H + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int DK, int DV>
+template <int DK, int DV, bool SEPV>
 cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
-  using Cf = Cfg<DK, DV>;
+  using Cf = Cfg<DK, DV, SEPV>;
   AttnParams p;
+  p.map = a.map;
   p.q = a.q;
   p.kv = a.kv;
+  p.v = a.v;
   p.idx = a.idx;
+  p.dense_rows = a.dense_rows;
+  p.kslots = a.idx != nullptr ? a.k : a.S;
   p.out = a.out;
   p.lse = a.lse;
   p.T = a.T;
@@ -623,7 +650,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   p.k = a.k;
   p.rows = a.B * a.T;
   p.nsplit = a.nsplit;
-  p.kc = ((a.k + a.nsplit - 1) / a.nsplit + kN - 1) / kN * kN;
+  p.kc = ((p.kslots + a.nsplit - 1) / a.nsplit + kN - 1) / kN * kN;
   p.scale_log2 = a.tau * 1.4426950408889634f;
   p.wait_ns = c.wait_ns;
   p.err = c.err;
@@ -636,11 +663,11 @@ cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, (uint64_t)rows * a.H, DK, (uint64_t)DK * 2, 128,
                     64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cf::ALLOC);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<DK, DV, SEPV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (e != cudaSuccess) return e;
   const long long ctas = rows * a.nsplit * Cf::NHALF;
-  sparse_attn_tc_kernel<DK, DV><<<(unsigned)ctas, kThreads, Cf::ALLOC, c.stream>>>(tm_q, p);
+  sparse_attn_tc_kernel<DK, DV, SEPV><<<(unsigned)ctas, kThreads, Cf::ALLOC, c.stream>>>(tm_q, p);
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.nsplit == 1) return e;
@@ -672,8 +699,9 @@ int attn_choose_nsplit(int rows, int H, int d_v, int k, int num_sms) {
 cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a) {
   if ((long long)a.B * a.T <= 0) return cudaSuccess;
   if (a.nsplit > 1 && a.part == nullptr) return cudaErrorInvalidValue;
-  if (a.d_k == 576 && a.d_v == 512) return launch_tc<576, 512>(c, a);
-  if (a.d_k == 80 && a.d_v == 64) return launch_tc<80, 64>(c, a);
+  const bool sepv = a.v != nullptr;
+  if (a.d_k == 576 && a.d_v == 512) return sepv ? launch_tc<576, 512, true>(c, a) : launch_tc<576, 512, false>(c, a);
+  if (a.d_k == 80 && a.d_v == 64) return sepv ? launch_tc<80, 64, true>(c, a) : launch_tc<80, 64, false>(c, a);
   return cudaErrorInvalidValue;
 }
 

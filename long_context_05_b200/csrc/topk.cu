@@ -310,12 +310,13 @@ __device__ void select_from_bin(const float* row, int n, int k, int32_t* out, un
   }
 }
 
-__device__ __forceinline__ void row_setup(const TopkArgs& a, int r, int* b, int* t, int* n, const float** row,
-                                          int32_t** out) {
+// Row r of the launch: sequence b, query t, n = pos(t) + 1 visible keys.
+__device__ __forceinline__ void row_setup(const TopkArgs& a, int r, DevErr* err, int* b, int* t, int* n,
+                                          const float** row, int32_t** out) {
   *b = r / a.q_count;
   const int i = r - *b * a.q_count;
   *t = a.q_begin + i;
-  *n = a.S - a.T + *t + 1;
+  *n = a.kv.len(*b, err, ERR_SITE_TOPK) - a.T + *t + 1;
   *row = a.scores + (size_t)r * a.ld;
   *out = a.idx + ((size_t)*b * a.T + *t) * a.k;
 }
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevEr
   int b, t, n;
   const float* row;
   int32_t* out;
-  row_setup(a, blockIdx.x, &b, &t, &n, &row, &out);
+  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
   const int k = a.k;
   if (n <= k) {
     for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
@@ -463,13 +464,13 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevEr
 // Workspace per row: hist[kBins] u32.  Kernel 1 adds each segment's histogram;
 // kernel 2 (one block per row) finds the bin and runs steps 2-3.
 
-__global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist, int hstride) {
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist, int hstride, DevErr* err) {
   __shared__ unsigned int hist[kBins];
   const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
   int b, t, n;
   const float* row;
   int32_t* out;
-  row_setup(a, r, &b, &t, &n, &row, &out);
+  row_setup(a, r, err, &b, &t, &n, &row, &out);
   if (n <= a.k) return;
   for (int x = threadIdx.x; x < kBins; x += kThreads) hist[x] = 0u;
   __syncthreads();
@@ -492,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs 
   int b, t, n;
   const float* row;
   int32_t* out;
-  row_setup(a, r, &b, &t, &n, &row, &out);
+  row_setup(a, r, err, &b, &t, &n, &row, &out);
   const int k = a.k;
   if (n <= k) return;
   unsigned int* w = ws + (size_t)r * kWsRowWords;
@@ -588,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_seg_final_kernel(TopkArgs a,
   int b, t, n;
   const float* row;
   int32_t* out;
-  row_setup(a, blockIdx.x, &b, &t, &n, &row, &out);
+  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
   const int k = a.k;
   if (n <= k) {
     for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
@@ -625,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_seg_select_kernel(TopkArgs a
   int b, t, n;
   const float* row;
   int32_t* out;
-  row_setup(a, blockIdx.x, &b, &t, &n, &row, &out);
+  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
   const int k = a.k;
   if (n <= k) {
     for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
@@ -640,6 +641,61 @@ __global__ void __launch_bounds__(kThreads, 2) topk_seg_select_kernel(TopkArgs a
   const unsigned int inbin = B < (unsigned)kBins ? sm.hist[B] : 0u;
   __syncthreads();
   select_from_bin(row, n, k, out, B, above, inbin, sm, err);
+}
+
+// Merge of candidate lists (key-split rows): row r's candidates are
+// nparts lists of k (score, global index) pairs, index -1 = empty.  Keeps the
+// k best by (score descending, index ascending) -- the top-k of the whole row
+// when each list is the top-k of a disjoint key range -- as global indices,
+// and, with idx_local set, the same selection as indices local to the key
+// range [local_begin, local_begin + local_count) (-1 outside it).
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_merge_kernel(const float* cand_scores, const int32_t* cand_idx, int rows, int nparts, int k, int32_t* idx,
+                      int local_begin, int local_count, int32_t* idx_local, DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int r = blockIdx.x;
+  int32_t* out = idx + (size_t)r * k;
+  if (threadIdx.x == 0) {
+    sm.ncand = 0;
+    sm.cnt = 0;
+  }
+  __syncthreads();
+  for (int x = threadIdx.x; x < nparts * k; x += kThreads) {
+    const int part = x / k, j = x - part * k;
+    const size_t o = ((size_t)part * rows + r) * k + j;
+    const int gi = cand_idx[o];
+    if (gi >= 0) {
+      const int q = atomicAdd(&sm.ncand, 1);
+      if (q < kCap) {
+        sm.ck[q] = order_key(cand_scores[o]);
+        sm.ci[q] = gi;
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = min(sm.ncand, kCap);
+  const int keep = min(nc, k);
+  if (keep > 0) select_candidates(nc, 0u, 0u, 32, (unsigned int)keep, k, out, sm, err);
+  __syncthreads();
+  for (int x = keep + threadIdx.x; x < k; x += kThreads) out[x] = -1;
+  if (idx_local != nullptr) {
+    __syncthreads();
+    for (int x = threadIdx.x; x < k; x += kThreads) {
+      const int g = out[x];
+      idx_local[(size_t)r * k + x] = (g >= local_begin && g - local_begin < local_count) ? g - local_begin : -1;
+    }
+  }
+}
+
+// Rows that see at most k keys keep all of them: idx = 0..n-1, then -1.
+// No score is read.
+__global__ void topk_fill_kernel(TopkArgs a, DevErr* err) {
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
+  for (int x = threadIdx.x; x < a.k; x += blockDim.x) out[x] = x < n ? x : -1;
 }
 
 // Zero the first `words` words of each of `rows` rows of `stride` words.
@@ -660,6 +716,12 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
   if (rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(Smem);
   cudaError_t e;
+  if ((long long)a.S - a.T + a.q_begin + a.q_count <= a.k) {
+    // every row sees at most k keys whatever its sequence's length
+    topk_fill_kernel<<<rows, 256, 0, c.stream>>>(a, c.err);
+    note_launches(1);
+    return cudaGetLastError();
+  }
   // few long rows: split the histogram pass over several blocks per row
   const bool split =
       ws != nullptr && ws_bytes >= topk_workspace_bytes(rows) && topk_uses_workspace(rows, a.S, c.num_sms);
@@ -672,7 +734,7 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
   }
   unsigned int* w = static_cast<unsigned int*>(ws);
   topk_zero_kernel<<<64, 256, 0, c.stream>>>(w, rows, kWsRowWords, kWsKeys);
-  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, kWsRowWords);
+  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, kWsRowWords, c.err);
   topk_seg_collect_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, c.err);
   e = cudaFuncSetAttribute(topk_seg_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -685,13 +747,29 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
 
 namespace dsa {
 
+cudaError_t launch_topk_merge(const LaunchCtx& c, const float* cand_scores, const int32_t* cand_idx, int rows,
+                              int nparts, int k, int32_t* idx, int local_begin, int local_count,
+                              int32_t* idx_local) {
+  if (rows <= 0) return cudaSuccess;
+  if ((long long)nparts * k > kCap) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_merge_kernel<<<rows, kThreads, smem, c.stream>>>(cand_scores, cand_idx, rows, nparts, k, idx, local_begin,
+                                                        local_count, idx_local, c.err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+int topk_merge_max_candidates() { return kCap; }
+
 // Split path with a caller-provided histogram array (B * q_count * 2048
 // words): zero it, histogram each row over several blocks, select per row.
 cudaError_t launch_topk_split_into(const LaunchCtx& c, const TopkArgs& a, unsigned int* hist) {
   const int rows = a.B * a.q_count;
   if (rows <= 0) return cudaSuccess;
   topk_zero_kernel<<<64, 256, 0, c.stream>>>(hist, rows, kBins, kBins);
-  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, hist, kBins);
+  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, hist, kBins, c.err);
   const size_t smem = sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(topk_seg_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -28,6 +28,7 @@ EXPORTS = [
     "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk",
     "dsa_sparse_attn", "dsa_forward", "dsa_prefill", "dsa_decode", "dsa_get_device_error",
     "dsa_set_wait_timeout_us", "dsa_launch_count", "dsa_selftest_wait_timeout", "dsa_topk_static",
+    "dsa_dense_attn", "dsa_topk_candidates", "dsa_topk_merge", "dsa_attn_combine",
 ]
 
 
@@ -42,12 +43,16 @@ class Shape(ctypes.Structure):
         ("mode", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
         ("H_I", ctypes.c_int), ("D_I", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
         ("d_v", ctypes.c_int), ("k", ctypes.c_int), ("q_block", ctypes.c_int),
-        ("softmax_scale", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float), ("seqlens", ctypes.c_void_p), ("page_size", ctypes.c_int),
+        ("pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int), ("block_table", ctypes.c_void_p),
     ]
 
 
+INPUT_NAMES = ("q_I", "q_scale", "w", "k_I", "k_scale", "q", "kv", "v")
+
+
 class Inputs(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("q_I", "q_scale", "w", "k_I", "k_scale", "q", "kv")]
+    _fields_ = [(n, ctypes.c_void_p) for n in INPUT_NAMES]
 
 
 _lib = None
@@ -74,7 +79,15 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk_static.restype = i
         L.dsa_topk_static.argtypes = [sp, vp, i64, i, i, vp, vp]
         L.dsa_sparse_attn.restype = i
-        L.dsa_sparse_attn.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_sparse_attn.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_dense_attn.restype = i
+        L.dsa_dense_attn.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_topk_candidates.restype = i
+        L.dsa_topk_candidates.argtypes = [sp, vp, i64, vp, ctypes.c_int32, vp, vp, vp]
+        L.dsa_topk_merge.restype = i
+        L.dsa_topk_merge.argtypes = [sp, i, vp, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp]
+        L.dsa_attn_combine.restype = i
+        L.dsa_attn_combine.argtypes = [sp, i, vp, vp, vp, vp, vp]
         for fn in ("dsa_forward", "dsa_prefill", "dsa_decode"):
             getattr(L, fn).restype = i
             getattr(L, fn).argtypes = [sp, ctypes.POINTER(Inputs), vp, vp, vp, vp, sz, vp]
@@ -90,18 +103,41 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def make_shape(wl=None, mode=None, **kw) -> Shape:
-    """Shape from a Workload (long_context_05_b200.inputs) and/or keywords."""
+def make_shape(wl=None, mode=None, seqlens=None, block_table=None, page_size=0, num_pages=0, **kw) -> Shape:
+    """Shape from a Workload (long_context_05_b200.inputs) and/or keywords.
+
+    seqlens: int32 CUDA tensor [B] of per-sequence key counts (or None).
+    block_table: int32 CUDA tensor [B, pages_per_seq] for paged caches, with
+    page_size and num_pages.  The shape keeps references to both tensors, so
+    their device pointers stay valid while the shape is alive."""
     f = {n: 0 for n, _ in Shape._fields_}
     f["softmax_scale"] = 0.0
+    f["seqlens"] = None
+    f["block_table"] = None
     if wl is not None:
         for n in ("B", "T", "S", "H_I", "D_I", "H", "d_k", "d_v", "k", "q_block"):
             f[n] = getattr(wl, n)
         f["mode"] = DSA_DECODE if wl.decode else DSA_PREFILL
     if mode is not None:
         f["mode"] = mode
+    keep = []
+    if seqlens is not None:
+        _need(seqlens, torch.int32, "seqlens")
+        f["seqlens"] = seqlens.data_ptr()
+        keep.append(seqlens)
+    f["page_size"] = page_size
+    f["num_pages"] = num_pages
+    if isinstance(block_table, int):        # a raw device address (pages_per_seq in kw)
+        f["block_table"] = block_table
+    elif block_table is not None:
+        _need(block_table, torch.int32, "block_table")
+        f["block_table"] = block_table.data_ptr()
+        f["pages_per_seq"] = block_table.shape[-1]
+        keep.append(block_table)
     f.update(kw)
-    return Shape(**f)
+    sh = Shape(**f)
+    sh._keep = keep
+    return sh
 
 
 def _p(t):
@@ -168,26 +204,86 @@ def topk_static(shape: Shape, scores: torch.Tensor, q_begin: int, q_count: int,
     return idx
 
 
-def sparse_attn(shape: Shape, q, kv, idx, out, lse=None, ws=None):
-    """Step C: out [B, T, H, d_v] bf16 (+ lse [B, T, H] fp32)."""
+def sparse_attn(shape: Shape, q, kv, idx, out, lse=None, ws=None, v=None):
+    """Step C: out [B, T, H, d_v] bf16 (+ lse [B, T, H] fp32).  v: separate
+    values [.., d_v] bf16, or None for V = kv[..., :d_v]."""
     _need(q, torch.bfloat16, "q")
     _need(kv, torch.bfloat16, "kv")
     _need(idx, torch.int32, "idx")
     _need(out, torch.bfloat16, "out")
     if lse is not None:
         _need(lse, torch.float32, "lse")
+    if v is not None:
+        _need(v, torch.bfloat16, "v")
     _check("dsa_sparse_attn", lib().dsa_sparse_attn(
-        ctypes.byref(shape), _p(q), _p(kv), _p(idx), _p(out), _p(lse), _p(ws),
+        ctypes.byref(shape), _p(q), _p(kv), _p(v), _p(idx), _p(out), _p(lse), _p(ws),
         0 if ws is None else ws.numel(), _stream()))
     return out, lse
 
 
+def dense_attn(shape: Shape, q, kv, out, lse=None, ws=None, v=None):
+    """Dense causal attention over every visible key (no selection)."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv, torch.bfloat16, "kv")
+    _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    if v is not None:
+        _need(v, torch.bfloat16, "v")
+    _check("dsa_dense_attn", lib().dsa_dense_attn(
+        ctypes.byref(shape), _p(q), _p(kv), _p(v), _p(out), _p(lse), _p(ws),
+        0 if ws is None else ws.numel(), _stream()))
+    return out, lse
+
+
+def topk_candidates(shape: Shape, scores, idx, part_begin: int, cand_scores, cand_idx):
+    """(score, global index) pairs of a part's selection (key-split rows)."""
+    _need(scores, torch.float32, "scores")
+    _need(idx, torch.int32, "idx")
+    _need(cand_scores, torch.float32, "cand_scores")
+    _need(cand_idx, torch.int32, "cand_idx")
+    _check("dsa_topk_candidates", lib().dsa_topk_candidates(
+        ctypes.byref(shape), _p(scores), scores.shape[-1], _p(idx), part_begin, _p(cand_scores), _p(cand_idx),
+        _stream()))
+    return cand_scores, cand_idx
+
+
+def topk_merge(shape: Shape, cand_scores, cand_idx, idx, local_begin: int = 0, local_count: int = 0,
+               idx_local=None):
+    """Global top-k of [nparts, B*T, k] candidate lists (+ this part's local indices)."""
+    _need(cand_scores, torch.float32, "cand_scores")
+    _need(cand_idx, torch.int32, "cand_idx")
+    _need(idx, torch.int32, "idx")
+    if idx_local is not None:
+        _need(idx_local, torch.int32, "idx_local")
+    _check("dsa_topk_merge", lib().dsa_topk_merge(
+        ctypes.byref(shape), cand_scores.shape[0], _p(cand_scores), _p(cand_idx), _p(idx), local_begin,
+        local_count, _p(idx_local), _stream()))
+    return idx, idx_local
+
+
+def attn_combine(shape: Shape, o_parts, lse_parts, out, lse=None):
+    """Merge [nparts, ...] attention results over disjoint key subsets."""
+    _need(o_parts, torch.bfloat16, "o_parts")
+    _need(lse_parts, torch.float32, "lse_parts")
+    _need(out, torch.bfloat16, "out")
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    _check("dsa_attn_combine", lib().dsa_attn_combine(
+        ctypes.byref(shape), o_parts.shape[0], _p(o_parts), _p(lse_parts), _p(out), _p(lse), _stream()))
+    return out, lse
+
+
 def _inputs(inp: dict) -> Inputs:
+    """Inputs struct from a dict of tensors; "v" is optional (None = MLA form)."""
     for n, d in (("q_I", torch.uint8), ("q_scale", torch.float32), ("w", torch.float32),
                  ("k_I", torch.uint8), ("k_scale", torch.float32), ("q", torch.bfloat16),
                  ("kv", torch.bfloat16)):
         _need(inp[n], d, n)
-    return Inputs(*(inp[n].data_ptr() for n in ("q_I", "q_scale", "w", "k_I", "k_scale", "q", "kv")))
+    v = inp.get("v")
+    if v is not None:
+        _need(v, torch.bfloat16, "v")
+    return Inputs(*(inp[n].data_ptr() for n in INPUT_NAMES[:-1]), None if v is None else v.data_ptr())
 
 
 def forward(shape: Shape, inp: dict, out, lse, idx, ws, entry: str = "dsa_forward"):

@@ -164,24 +164,28 @@ def topk(scores, k: int, T: int | None = None, S: int | None = None) -> np.ndarr
 # ---------------------------------------------------------------------------
 
 
-def sparse_attention_row(q_t, kv, idx_t, d_v: int, tau: float):
+def sparse_attention_row(q_t, kv, idx_t, d_v: int, tau: float, v=None):
     """Attention of all heads of one query over the selected rows of kv.
 
     q_t [H, d_k], kv [S, d_k] (one row shared by every head; value = first d_v
     columns), idx_t [k] with -1 for empty slots (skipped; duplicates count as
     often as they appear).  For each head h:
         z_s = tau * q_t[h] . kv[s],   m = max_s z_s,   p_s = exp(z_s - m)
-        O[h] = sum_s p_s kv[s, :d_v] / sum_s p_s,      LSE[h] = m + ln sum_s p_s
+        O[h] = sum_s p_s V[s] / sum_s p_s,             LSE[h] = m + ln sum_s p_s
+    with V[s] = kv[s, :d_v] (MLA: the value is the cached latent), or, when a
+    separate value array v [S, d_v] is given, V[s] = v[s] (the same formula
+    with values kept apart from the keys).
     Returns (O [H, d_v], LSE [H]) in float64.
     """
     sel = np.asarray(idx_t)
     sel = sel[sel >= 0]
     K = np.asarray(kv[sel], np.float64)                       # [n, d_k]
+    V = K[:, :d_v] if v is None else np.asarray(v[sel], np.float64)
     z = tau * (np.asarray(q_t, np.float64) @ K.T)             # [H, n]
     m = z.max(axis=1, keepdims=True)
     p = np.exp(z - m)
     l = p.sum(axis=1, keepdims=True)
-    O = (p @ K[:, :d_v]) / l
+    O = (p @ V) / l
     lse = (m + np.log(l))[:, 0]
     return O, lse
 
@@ -196,15 +200,16 @@ def sparse_attention(q, kv, idx, d_v: int, tau: float):
     return O, L
 
 
-def dense_causal_attention_row(q_t, kv, pos: int, d_v: int, tau: float):
+def dense_causal_attention_row(q_t, kv, pos: int, d_v: int, tau: float, v=None):
     """Plain softmax attention of one query over every visible key 0..pos.
 
     Written without the selection machinery, as the textbook definition:
-    weights = exp(z - logsumexp(z)), O = weights @ V.  Used only to pin the
-    sparse path: with k >= pos + 1 every visible key is kept, so DSA must reduce
-    exactly to this.
+    weights = exp(z - logsumexp(z)), O = weights @ V, with V = kv[:, :d_v] or
+    the separate value array v.  It pins the sparse path (with k >= pos + 1
+    every visible key is kept, so DSA must reduce exactly to this) and is the
+    reference of the dense short-prefill form.
     """
-    V = np.asarray(kv[: pos + 1, :d_v], np.float64)
+    V = np.asarray((kv[:, :d_v] if v is None else v)[: pos + 1], np.float64)
     Kf = np.asarray(kv[: pos + 1], np.float64)
     out = np.empty((q_t.shape[0], d_v))
     lse = np.empty(q_t.shape[0])
@@ -214,6 +219,44 @@ def dense_causal_attention_row(q_t, kv, pos: int, d_v: int, tau: float):
         lse[h] = zmax + np.log(np.sum(np.exp(z - zmax)))
         out[h] = np.exp(z - lse[h]) @ V
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# one sequence's keys spread over several parts (key-split decode)
+# ---------------------------------------------------------------------------
+
+
+def topk_merge(cand_scores, cand_idx, k: int) -> np.ndarray:
+    """Top-k of the union of candidate lists (score, key index), index -1 =
+    empty slot: order by (score descending, index ascending), keep the first
+    min(k, n).  With disjoint key ranges and each list the top-k of its range
+    under the same order, this is the top-k of the whole row (an element of
+    the global top-k has fewer than k better elements globally, hence in its
+    own range).  Returns int64 [k] padded with -1."""
+    cs = np.asarray(cand_scores, np.float64).ravel()
+    ci = np.asarray(cand_idx, np.int64).ravel()
+    ok = ci >= 0
+    cs, ci = cs[ok], ci[ok]
+    order = np.lexsort((ci, -cs))
+    keep = ci[order[: min(k, ci.shape[0])]]
+    out = np.full(k, -1, dtype=np.int64)
+    out[: keep.shape[0]] = keep
+    return out
+
+
+def combine_partials(o_parts, lse_parts):
+    """Attention over a key set from its results over disjoint subsets:
+    with M = max_r LSE_r (parts with LSE = -inf, i.e. no key, are skipped),
+        O = sum_r e^(LSE_r - M) O_r / sum_r e^(LSE_r - M),
+        LSE = M + ln sum_r e^(LSE_r - M).
+    o_parts [P, H, d_v], lse_parts [P, H]; returns (O [H, d_v], LSE [H])."""
+    o = np.asarray(o_parts, np.float64)
+    ls = np.asarray(lse_parts, np.float64)
+    M = ls.max(axis=0)                                      # [H]
+    w = np.where(np.isfinite(ls), np.exp(ls - M[None, :]), 0.0)
+    den = w.sum(axis=0)
+    O = (w[:, :, None] * o).sum(axis=0) / den[:, None]
+    return O, M + np.log(den)
 
 
 # ---------------------------------------------------------------------------

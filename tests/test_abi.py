@@ -48,7 +48,20 @@ def test_host_side_calls_without_gpu(libpath):
     assert dsa.workspace_size(uns) == 0                     # D_I unsupported
     assert L.dsa_forward(None, None, None, None, None, None, 0, None) == 1
     assert L.dsa_indexer_scores(ctypes.byref(bad), None, None, None, None, None, 0, 1, None, 8, None) == 1
-    assert L.dsa_sparse_attn(ctypes.byref(uns), None, None, None, None, None, None, 0, None) == 2
+    assert L.dsa_sparse_attn(ctypes.byref(uns), None, None, None, None, None, None, None, 0, None) == 2
+    assert L.dsa_dense_attn(ctypes.byref(uns), None, None, None, None, None, None, 0, None) == 2
+    assert L.dsa_version() >= 200
+    # paged caches: the page size must be a multiple of 16 and the block table
+    # must cover S keys per sequence
+    paged = dict(B=2, T=1, S=1000, H_I=4, D_I=32, H=8, d_k=80, d_v=64, k=64, q_block=1, mode=dsa.DSA_DECODE)
+    fake_table = 1 << 20                                    # never dereferenced on the host
+    ok = dsa.make_shape(None, **paged, page_size=64, pages_per_seq=16, num_pages=40, block_table=fake_table)
+    assert dsa.workspace_size(ok) > 0
+    assert dsa.workspace_size(dsa.make_shape(None, **paged, page_size=40, pages_per_seq=25, num_pages=60,
+                                             block_table=fake_table)) == 0      # not a multiple of 16
+    assert dsa.workspace_size(dsa.make_shape(None, **paged, page_size=64, pages_per_seq=15, num_pages=40,
+                                             block_table=fake_table)) == 0      # 15 * 64 < S
+    assert dsa.workspace_size(dsa.make_shape(None, **paged, page_size=64, pages_per_seq=16, num_pages=40)) == 0
     assert L.dsa_launch_count() == 0
 
 

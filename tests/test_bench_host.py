@@ -41,9 +41,24 @@ def test_algorithmic_flops_per_pair(bench):
     peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 1000.0, "hbm_gbs": 1000.0}
     per_kernel = {"indexer": [1000.0], "topk": [1000.0], "sparse_attn": [1000.0]}  # 1 s each
     rep = bench.kernel_report(wl, per_kernel, 1, peaks, "test", sustained=True)
-    assert rep["indexer"]["achieved"] == pytest.approx(2 * 64 * 128 * 8_590_000_128 / 1e12)
+    # the first k rows keep every visible key: they are neither scored nor selected
+    scored = 8_590_000_128 - 2048 * 2049 // 2
+    assert bench.dense_rows(wl) == 2048 and bench.scored_pairs(wl) == scored
+    assert rep["indexer"]["achieved"] == pytest.approx(2 * 64 * 128 * scored / 1e12)
     assert rep["sparse_attn"]["achieved"] == pytest.approx(2 * 128 * (576 + 512) * 266_339_328 / 1e12)
-    assert rep["topk"]["achieved"] == pytest.approx(4 * 8_590_000_128 / 1e9)
+    assert rep["topk"]["achieved"] == pytest.approx(4 * scored / 1e9)
+
+
+def test_decode_indexer_is_reported_against_hbm(bench):
+    """In decode the indexer streams every key once: its roofline is HBM on
+    the k_I and k_scale bytes (8 x 131072 x 132 B = 138.4 MB for the 128K decode)."""
+    from long_context_05_b200.inputs import WORKLOADS
+    dec = WORKLOADS["decode_128k_b8"]
+    peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 1000.0, "hbm_gbs": 1000.0}
+    rep = bench.kernel_report(dec, {"indexer": [1.0], "topk": [1.0], "sparse_attn": [1.0]}, 1, peaks, "t", False)
+    assert rep["indexer"]["bound"] == "hbm" and rep["indexer"]["unit"] == "GB/s"
+    assert rep["indexer"]["work_per_step"] == pytest.approx(8 * 131072 * 132)
+    assert rep["sparse_attn"]["bound"] == "hbm"
 
 
 def test_traffic_reported_only_for_the_captured_source(bench):

@@ -2,8 +2,12 @@
 
 Every call goes through libdsa.so (ctypes binding); the oracle runs on CPU
 copies of the rows it checks.  Sizes: the tiny integer workload in full, small
-ragged shapes that span several tiles, the two decode workloads in full, and
-the prefill workloads at full size on stratified samples of query rows.
+ragged shapes that span several tiles, the two decode workloads in full (every
+row's whole score row element by element too), and the prefill workloads at
+full size on stratified samples of about 1,100-1,250 query rows each (the
+first 64, k-2..k+1, both sides of every query-block boundary, the last 64 and
+1,024 random rows), plus the whole score rows of 32 rows of one 4096-row
+block of the 128K prefill.  The sample size is in each test id.
 """
 import numpy as np
 import pytest
@@ -50,24 +54,28 @@ def _scores_for_rows(wl, inp, q_begin, q_count):
     return sc
 
 
-def _check_rows(wl, inp, outs, rows_by_b, exact, check_scores_too=True, tag=""):
-    """Oracle on the listed (b -> rows); compare scores, sets and outputs."""
+def _check_rows(wl, inp, outs, rows_by_b, exact, tag="", lengths=None, v=None):
+    """Oracle on the listed (b -> rows); compare index sets, outputs and LSE.
+    lengths: per-sequence key counts (None: all S); v: separate value array
+    [B, S, d_v] (float64) or None."""
     tau = _tau(wl)
-    shape = dsa.make_shape(wl)
     idx_gpu = outs.idx.cpu().numpy()
     out_gpu = outs.out.float().cpu().numpy()
     lse_gpu = outs.lse.cpu().numpy()
+    stats = P.ErrStats()
     for b, rows in rows_by_b.items():
         seq = P.OracleSeq(inp, b)
+        L = None if lengths is None else int(lengths[b])
         for t in rows:
             what = f"{tag} b={b} t={t}"
-            sc, idx_o = P.oracle_select(seq, wl, t)
+            sc, idx_o = P.oracle_select(seq, wl, t, L)
             P.check_selection(idx_gpu[b, t], idx_o, sc, exact, what)
             # end to end: oracle attention over the GPU's (validated) selection
-            o_g, lse_g = P.oracle_attn(seq, wl, t, tau, idx_gpu[b, t])
-            P.check_attention(out_gpu[b, t], o_g, what)
+            o_g, lse_g = P.oracle_attn(seq, wl, t, tau, idx_gpu[b, t], None if v is None else v[b])
+            stats.add(P.check_attention(out_gpu[b, t], o_g, what))
             assert np.allclose(lse_gpu[b, t], lse_g, atol=2e-3, rtol=1e-4), what
-    return True
+    print(stats.line(tag))
+    return stats
 
 
 # ----------------------------------------------------------------- tiny, exact
@@ -181,19 +189,62 @@ def test_decode_workloads_full(name):
     _check_rows(wl, inp, outs, {b: [0] for b in range(wl.B)}, exact=False, tag=name)
 
 
-@pytest.mark.parametrize("name,n_random", [("prefill_8k", 96), ("prefill_128k", 24)])
-def test_prefill_workloads_sampled(name, n_random):
+@pytest.mark.parametrize("name", ["decode_32k_b32", "decode_128k_b8"])
+def test_decode_indexer_scores_every_row_in_full(name):
+    """Every decode row's whole score row (32768 or 131072 entries), element by
+    element, in the launch configuration dsa_forward uses for decode (short key
+    runs per work item, double-buffered query tiles)."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, "cuda")
+    sc = _scores_for_rows(wl, inp, 0, 1).cpu().numpy()
+    for b in range(wl.B):
+        seq = P.OracleSeq(inp, b)
+        qd, w, _ = seq.query(0)
+        ref = O.indexer_row(qd, w, seq.kd, wl.S - 1)
+        P.check_scores(sc[b], ref, P.score_abs_scale(seq, wl, 0), False, f"{name} b={b}")
+
+
+# stratified samples of the prefill workloads: about 1.1-1.3K rows each
+PREFILL_SAMPLES = {name: P.sample_rows(WORKLOADS[name], 1024) for name in ("prefill_8k", "prefill_128k")}
+
+
+@pytest.mark.parametrize("name", list(PREFILL_SAMPLES),
+                         ids=[f"{n}-{len(r)}rows" for n, r in PREFILL_SAMPLES.items()])
+def test_prefill_workloads_sampled(name):
     wl = WORKLOADS[name]
     inp = make_inputs(wl, "cuda")
     outs = _run_forward(wl, inp)
-    rows = P.sample_rows(wl, n_random)
-    if name == "prefill_128k":
-        rows = [r for r in rows if r < 16 or r % 5 == 0 or r >= wl.T - 16]
+    rows = PREFILL_SAMPLES[name]
+    assert len(rows) >= 1000
     _check_rows(wl, inp, outs, {0: rows}, exact=False, tag=name)
     # rows with fewer visible keys than k keep all of them (dense)
     idx = outs.idx[0, : wl.k].cpu().numpy()
     for t in (0, 1, 100, wl.k - 1):
         assert sorted(idx[t][idx[t] >= 0]) == list(range(t + 1))
+
+
+def test_prefill_128k_indexer_block_scores():
+    """Whole score rows of 32 rows of one 4096-row query block of the 128K
+    prefill (the launch configuration of the benchmark: a full block, paired
+    key tiles, 16-query items), element by element: the first and last rows
+    of the block, rows on both sides of item (16-row) boundaries, random
+    rows."""
+    wl = WORKLOADS["prefill_128k"]
+    inp = make_inputs(wl, "cuda")
+    q0 = 16 * wl.q_block                   # rows 65536 .. 69631
+    sc = _scores_for_rows(wl, inp, q0, wl.q_block)
+    rng = np.random.default_rng(3)
+    picks = sorted(set([0, 1, 15, 16, 17, 2047, 2048, wl.q_block - 2, wl.q_block - 1] +
+                       rng.integers(0, wl.q_block, 23).tolist()))
+    seq = P.OracleSeq(inp, 0)
+    for i in picks:
+        t = q0 + i
+        row = sc[i].cpu().numpy()
+        qd, w, _ = seq.query(t)
+        ref = O.indexer_row(qd, w, seq.kd, t)
+        P.check_scores(row, ref, P.score_abs_scale(seq, wl, t), False, f"prefill_128k block t={t}")
+        assert np.all(np.isnan(row[t + 1: wl.S])), "wrote past the causal limit"
+    assert len(picks) >= 30
 
 
 # ----------------------------------------------------------------- errors

@@ -231,6 +231,24 @@ def test_attention_equal_logits_mean():
     assert np.allclose(lse, np.log(4.0))
 
 
+def test_attention_separate_values_single_key_and_mean():
+    """With values kept apart from the keys, one selected key returns its value
+    row exactly and equal logits return the mean of the selected value rows;
+    the key rows' own leading columns must play no part."""
+    rng = np.random.default_rng(5)
+    kv = rng.standard_normal((10, 12)); v = rng.standard_normal((10, 6))
+    q = rng.standard_normal((3, 12))
+    out, lse = O.sparse_attention_row(q, kv, np.array([-1, 4, -1]), d_v=6, tau=0.5, v=v)
+    assert np.array_equal(out, np.broadcast_to(v[4], (3, 6)))
+    assert np.allclose(lse, 0.5 * q @ kv[4])
+    sel = np.array([0, 3, 3, 8])
+    out, lse = O.sparse_attention_row(np.zeros((2, 12)), kv, sel, d_v=6, tau=1.0, v=v)
+    assert np.allclose(out, v[sel].mean(0), rtol=0, atol=1e-15)
+    assert np.allclose(lse, np.log(4.0))
+    od, ld = O.dense_causal_attention_row(np.zeros((2, 12)), kv, 4, 6, 1.0, v=v)
+    assert np.allclose(od, v[:5].mean(0), rtol=0, atol=1e-15) and np.allclose(ld, np.log(5.0))
+
+
 def test_attention_permutation_invariance_and_lse():
     rng = np.random.default_rng(6)
     kv = rng.standard_normal((50, 24)); q = rng.standard_normal((4, 24))
@@ -240,6 +258,34 @@ def test_attention_permutation_invariance_and_lse():
     assert np.allclose(o1, o2, atol=1e-14) and np.allclose(l1, l2, atol=1e-14)
     z = 0.2 * q @ kv[sel].T
     assert np.allclose(np.exp(z - l1[:, None]).sum(1), 1.0, atol=1e-14)
+
+
+def test_topk_merge_of_range_winners_equals_whole_row():
+    """The top-k of a row equals the merge of the top-k of its disjoint key
+    ranges, ties included (integer scores with large tie groups)."""
+    rng = np.random.default_rng(11)
+    for n, k, parts in ((1000, 64, 2), (3000, 512, 4), (257, 300, 3)):
+        row = rng.integers(-4, 5, n).astype(np.float64)
+        ref = O.topk_row(row, k)
+        bounds = np.linspace(0, n, parts + 1).astype(int)
+        cs, ci = [], []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            loc = O.topk_row(row[a:b], k)
+            ci.append(np.where(loc >= 0, loc + a, -1))
+            cs.append(np.where(loc >= 0, row[a + np.maximum(loc, 0)], 0.0))
+        assert np.array_equal(O.topk_merge(np.stack(cs), np.stack(ci), k), ref)
+
+
+def test_combine_partials_equals_attention_over_the_union():
+    rng = np.random.default_rng(12)
+    kv = rng.standard_normal((200, 24)); q = rng.standard_normal((3, 24)) * 2
+    sel = rng.choice(200, 60, replace=False)
+    o_all, l_all = O.sparse_attention_row(q, kv, sel, 16, 0.3)
+    parts = [sel[:10], sel[10:45], sel[45:], np.array([-1, -1])]      # the last part is empty
+    res = [O.sparse_attention_row(q, kv, s_, 16, 0.3) if (s_ >= 0).any()
+           else (np.zeros((3, 16)), np.full(3, -np.inf)) for s_ in parts]
+    o, l = O.combine_partials(np.stack([r[0] for r in res]), np.stack([r[1] for r in res]))
+    assert np.max(np.abs(o - o_all)) < 1e-12 and np.max(np.abs(l - l_all)) < 1e-12
 
 
 def test_sparse_equals_dense_when_k_covers_context():

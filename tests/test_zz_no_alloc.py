@@ -3,8 +3,12 @@
 It must select exactly what dsa_topk selects (integer index sets, so the
 tolerance is equality of the sorted sets), on two calls in a row: the second
 call reuses the library's fixed histogram array after the first, so any count
-left behind by the first call would change its answer.  The file is named to
-run last, after the other GPU tests have used the library on the same device.
+left behind by the first call would change its answer.  Rows of each call are
+also checked against the FP64 oracle's selection (the scores are FP32 values
+that both sides compare as they are), including the few-levels rows whose
+tie group at the k-th key is larger than the shared-memory candidate buffer.
+The file is named to run last, after the other GPU tests have used the
+library on the same device.
 """
 import ctypes
 
@@ -13,6 +17,7 @@ import pytest
 import torch
 
 from long_context_05_b200 import dsa
+from oracle import dsa_oracle as O
 
 DSA_ERR_WORKSPACE = 3
 MAX_ROWS = 64  # DSA_TOPK_STATIC_MAX_ROWS in include/dsa.h
@@ -77,3 +82,10 @@ def test_static_topk_matches_topk_twice(B, T, S, q_begin, q_count, k):
         n = S - T + q_begin + np.arange(q_count) + 1
         filled = (o.cpu().numpy() >= 0).sum(-1)
         assert (filled == np.minimum(n, k)[None, :]).all(), f"call {call}"
+        # against the oracle: the first, a middle and the last row of the call
+        og = o.cpu().numpy()
+        scn = sc.cpu().numpy()
+        for r in sorted({0, rows // 2, rows - 1}):
+            b, i = divmod(r, q_count)
+            ref = O.topk_row(scn[r, : n[i]].astype(np.float64), k)
+            assert sorted(og[b, i][og[b, i] >= 0].tolist()) == sorted(ref[ref >= 0].tolist()), (call, r)
