@@ -215,11 +215,18 @@ class DsaRunner:
         self.ws = dsa.alloc_workspace(self.shape)
         self.outs = dsa.alloc_outputs(wl)
         self.ld = (wl.S + 63) // 64 * 64
-        nscore = wl.B * self.rows_per_block() * self.ld * 4
-        self.scores = self.ws[:nscore].view(torch.float32).view(-1, self.ld)
-        # the top-k's scratch (histograms of the split path for few long
-        # rows) follows the scores, 256-byte aligned, as in dsa_forward
-        self.topk_ws = self.ws[(nscore + 255) // 256 * 256:]
+        if wl.decode:
+            # decode scores its rows into the workspace's score tile; the
+            # top-k's scratch (histograms of the split path for few long
+            # rows) follows it, 256-byte aligned, as in dsa_forward
+            nscore = wl.B * self.rows_per_block() * self.ld * 4
+            self.scores = self.ws[:nscore].view(torch.float32).view(-1, self.ld)
+            self.topk_ws = self.ws[(nscore + 255) // 256 * 256:]
+        else:
+            # prefill selects through dsa_select (its own use of the
+            # workspace); the index fill of the dense rows reads no score
+            self.scores = torch.zeros(1, self.ld, dtype=torch.float32, device="cuda")
+            self.topk_ws = None
         self.stream = torch.cuda.current_stream()
 
     def rows_per_block(self):
@@ -240,15 +247,25 @@ class DsaRunner:
             return e
 
         dr = dense_rows(wl)
+        sel = "select" if not wl.decode else "topk"
         if dr:
             # rows that keep all their visible keys: the index fill only
             e0 = mark()
             d.topk(self.shape, self.scores, 0, dr, o.idx, self.topk_ws)
             e1 = mark()
             if ev is not None:
-                ev.append(("topk", e0, e1))
+                ev.append((sel, e0, e1))
         for q0 in range(dr, wl.T, qb):
             cnt = min(qb, wl.T - q0)
+            if not wl.decode:
+                # prefill: steps A and B of the block in one call (no score
+                # tile over long contexts)
+                e0 = mark()
+                d.select(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, o.idx, self.ws)
+                e1 = mark()
+                if ev is not None:
+                    ev.append(("select", e0, e1))
+                continue
             e0 = mark()
             d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, self.scores)
             e1 = mark()
@@ -271,11 +288,13 @@ class DsaRunner:
             d.sparse_attn(self.shape, i["q"], i["kv"], o.idx, o.out, o.lse, self.ws)
             return
         dr = dense_rows(wl)
-        if dr and name == "topk":
+        if dr and name in ("topk", "select"):
             d.topk(self.shape, self.scores, 0, dr, o.idx, self.topk_ws)
         for q0 in range(dr, wl.T, qb):
             cnt = min(qb, wl.T - q0)
-            if name == "indexer":
+            if name == "select":
+                d.select(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, o.idx, self.ws)
+            elif name == "indexer":
                 d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt,
                                  self.scores)
             else:
@@ -405,6 +424,11 @@ def kernel_report(wl, per_kernel, steps, peaks, peak_src, sustained):
                     (wl.B * wl.S * (wl.D_I + 4) / 1e9, "GB/s", "hbm", peaks["hbm_gbs"],
                      f"hbm, k_I + k_scale bytes ({peak_src})")),
         "topk": (4.0 * ip / 1e9, "GB/s", "hbm", peaks["hbm_gbs"], f"hbm ({peak_src})"),
+        # prefill: the indexer and the selection fused (dsa_select); its work
+        # is the indexer's, so the fraction is a lower bound on the indexer's
+        "select": (2.0 * wl.H_I * wl.D_I * ip / 1e12, "TFLOP/s", "tensor", bf16 * FP8_PER_BF16,
+                   f"indexer FLOP over the fused indexer + top-k time; fp8 = {kind} bf16 x {FP8_PER_BF16:g} "
+                   f"({peak_src})"),
         "sparse_attn": ((2.0 * wl.H * (wl.d_k + wl.d_v) * ap / 1e12, "TFLOP/s", "tensor", bf16,
                          f"bf16 {kind} ({peak_src})") if not wl.decode else
                         (2.0 * wl.d_k * ap / 1e9, "GB/s", "hbm", peaks["hbm_gbs"], f"hbm, gathered KV bytes ({peak_src})")),

@@ -170,6 +170,27 @@ DSA_API dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
                     int64_t ld_scores, int q_begin, int q_count, int32_t* idx,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* Steps A and B together for queries [q_begin, q_begin + q_count): writes the
+ * selection idx[b, t, 0..k) as dsa_topk does (ties to the lower index, -1
+ * after the last).  ws: dsa_workspace_size(shape) bytes.
+ * In prefill over long contexts (S >= 32768, S a multiple of 16, contiguous
+ * caches) the query block's score matrix is never stored (the pages ask that
+ * the selection be cache-aware and stay on the device: sider.ai blog on
+ * DeepSeek Sparse Attention, "Uyarilar"): the
+ * indexer scores every 16th key, a per-row radix select on that sample gives
+ * a threshold expected to admit about 2k keys, the indexer then scores every
+ * key and keeps only (score, index) pairs at or above the row's threshold
+ * (at most 8192 per row), and the top k are selected exactly among them.  A
+ * row left with fewer than k candidates, or more than the list holds, is
+ * scored again in full into a small tile and selected from it, so the result
+ * is the same exact top-k on any input (up to 64 such rows per query block;
+ * beyond that DSA_ERR_DEVICE_BOUNDS is reported).  Otherwise the block's
+ * scores go through the workspace as dsa_indexer_scores + dsa_topk. */
+DSA_API dsa_status dsa_select(const dsa_shape* shape, const uint8_t* q_I,
+                      const float* q_scale, const float* w, const uint8_t* k_I,
+                      const float* k_scale, int q_begin, int q_count,
+                      int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
 /* Step B without any allocation (an addition of this library; the sparse
  * attention papers have no counterpart).  Same arguments, output and error
  * checks as dsa_topk, minus the workspace: the per-row histograms of the split
@@ -291,6 +312,51 @@ DSA_API dsa_status dsa_topk_merge(const dsa_shape* shape, int nparts,
 DSA_API dsa_status dsa_attn_combine(const dsa_shape* shape, int nparts,
                             const uint16_t* o_parts, const float* lse_parts,
                             uint16_t* out, float* lse, void* stream);
+
+/* ---- Training the indexer (kernel level) ----------------------------------
+ * tenelement.pl, "DeepSeek V3.2-Exp Cuts Long-Context Costs ...", section
+ * "Proces Treningu DSA: Od Warm-up do Sparsity": a warm-up in which the
+ * indexer learns the dense model's attention distribution through a KL
+ * divergence with the main model frozen, then a sparse stage over the top-k
+ * set; the indexer's gradients stay apart from the main language loss.
+ * Readings (the pages give no formula): the target of query t is the main
+ * attention's weights summed over heads and divided by H; the loss is
+ * KL(target || softmax(I[t, .])) over the visible keys (idx NULL: warm-up)
+ * or over the selected set idx[b, t, :] (sparse stage); the target is a
+ * constant.  Rows are queries [q_begin, q_begin + q_count) of every
+ * sequence, row r = b * q_count + i of the [rows, ld] FP32 arrays. */
+
+/* target[r, s] = (1/H) sum_h exp(tau q[b,t,h] . kv[b,s] - lse[b,t,h]) for
+ * every visible key s (idx NULL) or every key of the set; lse [B, T, H] is
+ * the main attention's natural log-sum-exp over the same keys (dsa_dense_attn
+ * or dsa_sparse_attn output).  Other entries are left untouched.
+ * d_k must be 576 (the MLA row). */
+DSA_API dsa_status dsa_kl_target(const dsa_shape* shape, const uint16_t* q,
+                         const uint16_t* kv, const float* lse, const int32_t* idx,
+                         int q_begin, int q_count, float* target, int64_t ld,
+                         void* stream);
+
+/* Per row: loss[r] = KL(target || softmax(I)) over the set, and
+ * grad[r, s] = softmax(I)_s - target[r, s] for keys of the set, 0 for other
+ * visible keys.  scores: the indexer scores as dsa_indexer_scores writes
+ * them for the same rows. */
+DSA_API dsa_status dsa_indexer_kl(const dsa_shape* shape, const float* scores,
+                          const float* target, int64_t ld, const int32_t* idx,
+                          int q_begin, int q_count, float* grad, float* loss,
+                          void* stream);
+
+/* Gradients of sum_s grad[r, s] I[t, s] with respect to the dequantised
+ * indexer inputs (FP32): dq [B, T, H_I, D_I] and dw [B, T, H_I] (rows of the
+ * launch written), dk [B, S, D_I] accumulated into (+=; zero it first; paged
+ * caches: the pool layout).  idx: the set whose keys carry gradient (NULL:
+ * every visible key).  Supported (H_I, D_I): (64, 128), (32, 128),
+ * (16, 128), (64, 64), (32, 64). */
+DSA_API dsa_status dsa_indexer_backward(const dsa_shape* shape, const uint8_t* q_I,
+                                const float* q_scale, const float* w,
+                                const uint8_t* k_I, const float* k_scale,
+                                const float* grad, int64_t ld, const int32_t* idx,
+                                int q_begin, int q_count, float* dq, float* dw,
+                                float* dk, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_BOUNDS

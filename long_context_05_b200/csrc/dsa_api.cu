@@ -125,9 +125,28 @@ float tau_of(const dsa_shape* s) {
   return s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / sqrtf((float)s->d_k);
 }
 
+// Selection without a score tile: prefill over long contexts with a
+// contiguous key cache (the sample reads every kSampleStride-th cache row).
+constexpr int kSampleStride = 16;
+constexpr int kRepairRows = 64;   // rows of one block that can fall back to a materialised score row
+
+bool fused_select(const dsa_shape* s) {
+  return s->mode == DSA_PREFILL && s->page_size == 0 && s->S % kSampleStride == 0 &&
+         s->S >= 4 * topk_cand_cap();
+}
+
 // Workspace layout (each region 256-byte aligned):
-//   [scores: B * q_rows * ld floats][attention split partials][top-k histograms]
+//   [score tile, or the fused selection's regions][attention split partials]
+//   [top-k histograms]
+// The fused selection's regions, for R = B * q_rows rows: the key-sample
+// tile [R, ld_s] FP32, thresholds, candidate counts and repair slots [R],
+// candidate keys and indices [R, cap], the repair list and its count, and
+// the repair tile [kRepairRows, ld] FP32.
 struct WsLayout {
+  bool fused;
+  size_t sample_off, thr_off, cnt_off, slot_off, ckey_off, cidx_off, fail_off, nfail_off, repair_off;
+  int64_t ld_s;
+  int cap;
   size_t scores_off, scores_bytes;
   size_t part_off, part_bytes;
   size_t topk_off, topk_bytes;
@@ -140,7 +159,25 @@ WsLayout ws_layout(const dsa_shape* s, int num_sms) {
   WsLayout L;
   L.q_rows = s->mode == DSA_DECODE ? s->T : q_block_of(s);
   L.scores_off = 0;
-  L.scores_bytes = round_up((size_t)s->B * L.q_rows * scores_ld(s) * sizeof(float), 256);
+  L.fused = fused_select(s);
+  L.cap = topk_cand_cap();
+  L.ld_s = (int64_t)round_up((size_t)(s->S / kSampleStride), 64);
+  if (L.fused) {
+    const size_t R = (size_t)s->B * L.q_rows;
+    size_t o = 0;
+    L.sample_off = o; o += round_up(R * L.ld_s * sizeof(float), 256);
+    L.thr_off = o; o += round_up(R * 4, 256);
+    L.cnt_off = o; o += round_up(R * 4, 256);
+    L.slot_off = o; o += round_up(R * 4, 256);
+    L.ckey_off = o; o += round_up(R * L.cap * 4, 256);
+    L.cidx_off = o; o += round_up(R * L.cap * 4, 256);
+    L.fail_off = o; o += round_up(kRepairRows * 4, 256);
+    L.nfail_off = o; o += 256;
+    L.repair_off = o; o += round_up((size_t)kRepairRows * scores_ld(s) * sizeof(float), 256);
+    L.scores_bytes = o;
+  } else {
+    L.scores_bytes = round_up((size_t)s->B * L.q_rows * scores_ld(s) * sizeof(float), 256);
+  }
   L.nsplit = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->d_v, s->k, num_sms) : 1;
   // dense attention (dsa_dense_attn) splits a decode row's S keys instead
   L.nsplit_dense = s->mode == DSA_DECODE ? attn_choose_nsplit(s->B * s->T, s->H, s->d_v, s->S, num_sms) : 1;
@@ -166,8 +203,9 @@ dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR
 dsa_status run_indexer(const LaunchCtx& c, const dsa_shape* s, const uint8_t* q_I, const float* q_scale,
                        const float* w, const uint8_t* k_I, const float* k_scale, int q_begin, int q_count,
                        float* scores, int64_t ld) {
-  IndexerArgs a;
+  IndexerArgs a = {};
   a.kv = kv_map(s);
+  a.kstride = 1;
   a.q_I = q_I; a.q_scale = q_scale; a.w = w; a.k_I = k_I; a.k_scale = k_scale;
   a.scores = scores; a.ld = ld;
   a.B = s->B; a.T = s->T; a.S = s->S; a.H_I = s->H_I; a.D_I = s->D_I;
@@ -183,6 +221,84 @@ dsa_status run_topk(const LaunchCtx& c, const dsa_shape* s, const float* scores,
   a.B = s->B; a.T = s->T; a.S = s->S; a.k = s->k;
   a.q_begin = q_begin; a.q_count = q_count;
   return from_cuda(launch_topk(c, a, ws, ws_bytes));
+}
+
+// Steps A and B for query rows [q0, q0 + cnt) (cnt <= q_rows) without the
+// score tile: key sample -> thresholds -> candidates -> exact selection ->
+// repair of the rows that fell short or overflowed.
+dsa_status run_select_fused(const LaunchCtx& c, const dsa_shape* s, const WsLayout& L, char* ws, const uint8_t* q_I,
+                            const float* q_scale, const float* w, const uint8_t* k_I, const float* k_scale, int q0,
+                            int cnt, int32_t* idx) {
+  float* sample = reinterpret_cast<float*>(ws + L.sample_off);
+  unsigned int* thr = reinterpret_cast<unsigned int*>(ws + L.thr_off);
+  unsigned int* ccnt = reinterpret_cast<unsigned int*>(ws + L.cnt_off);
+  int* slot = reinterpret_cast<int*>(ws + L.slot_off);
+  unsigned int* ckey = reinterpret_cast<unsigned int*>(ws + L.ckey_off);
+  int32_t* cidx = reinterpret_cast<int32_t*>(ws + L.cidx_off);
+  int* fail = reinterpret_cast<int*>(ws + L.fail_off);
+  unsigned int* nfail = reinterpret_cast<unsigned int*>(ws + L.nfail_off);
+  float* repair = reinterpret_cast<float*>(ws + L.repair_off);
+  IndexerArgs ia = {};
+  ia.kv = kv_map(s);
+  ia.kstride = 1;
+  ia.q_I = q_I; ia.q_scale = q_scale; ia.w = w; ia.k_I = k_I; ia.k_scale = k_scale;
+  ia.B = s->B; ia.T = s->T; ia.S = s->S; ia.H_I = s->H_I; ia.D_I = s->D_I;
+  ia.q_begin = q0; ia.q_count = cnt;
+  TopkArgs ta;
+  ta.kv = kv_map(s);
+  ta.scores = nullptr; ta.ld = 0; ta.idx = idx;
+  ta.B = s->B; ta.T = s->T; ta.S = s->S; ta.k = s->k;
+  ta.q_begin = q0; ta.q_count = cnt;
+  cudaError_t e;
+  // 1. scores of every kSampleStride-th key, when some row sees more keys
+  //    than its candidate list holds
+  const bool long_rows = (long long)s->S - s->T + q0 + cnt > L.cap;
+  if (long_rows) {
+    IndexerArgs sa = ia;
+    sa.kstride = kSampleStride;
+    sa.scores = sample;
+    sa.ld = L.ld_s;
+    if ((e = launch_indexer(c, sa)) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  // 2. per-row thresholds (about 2k expected candidates), counts cleared
+  if ((e = launch_topk_threshold(c, ta, sample, L.ld_s, kSampleStride, 2 * s->k, thr, ccnt, slot, nfail)) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  // 3. every key scored, candidates appended
+  IndexerArgs ca = ia;
+  ca.thr = thr;
+  ca.cand_key = ckey;
+  ca.cand_idx = cidx;
+  ca.cand_cnt = ccnt;
+  ca.cand_cap = L.cap;
+  if ((e = launch_indexer(c, ca)) != cudaSuccess) return DSA_ERR_CUDA;
+  // 4. exact selection among the candidates
+  if ((e = launch_topk_cand_select(c, ta, ckey, cidx, ccnt, L.cap, slot, fail, nfail, kRepairRows)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  // 5. repair (both launches return at once when no row was listed)
+  IndexerArgs ra = ia;
+  ra.row_slot = slot;
+  ra.scores = repair;
+  ra.ld = scores_ld(s);
+  if ((e = launch_indexer(c, ra)) != cudaSuccess) return DSA_ERR_CUDA;
+  TopkArgs rt = ta;
+  if ((e = launch_topk_repair(c, rt, repair, scores_ld(s), fail, nfail, kRepairRows)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+// Steps A and B for rows [q0, q0 + cnt) through the workspace: fused when it
+// applies, else the score tile and dsa_topk's selection.
+dsa_status run_select(const LaunchCtx& c, const dsa_shape* s, const WsLayout& L, void* ws, const uint8_t* q_I,
+                      const float* q_scale, const float* w, const uint8_t* k_I, const float* k_scale, int q0, int cnt,
+                      int32_t* idx) {
+  if (L.fused) return run_select_fused(c, s, L, static_cast<char*>(ws), q_I, q_scale, w, k_I, k_scale, q0, cnt, idx);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + L.scores_off);
+  const int64_t ld = scores_ld(s);
+  dsa_status st = run_indexer(c, s, q_I, q_scale, w, k_I, k_scale, q0, cnt, scores, ld);
+  if (st != DSA_OK) return st;
+  return run_topk(c, s, scores, ld, q0, cnt, idx, L.topk_bytes ? static_cast<char*>(ws) + L.topk_off : nullptr,
+                  L.topk_bytes);
 }
 
 // idx null: dense causal attention of every row; otherwise rows t <
@@ -274,6 +390,24 @@ dsa_status dsa_topk(const dsa_shape* s, const float* scores, int64_t ld_scores, 
   return run_topk(c, s, scores, ld_scores, q_begin, q_count, idx, ws, ws_bytes);
 }
 
+dsa_status dsa_select(const dsa_shape* s, const uint8_t* q_I, const float* q_scale, const float* w,
+                      const uint8_t* k_I, const float* k_scale, int q_begin, int q_count, int32_t* idx, void* ws,
+                      size_t ws_bytes, void* stream) {
+  dsa_status st = check_shape(s);
+  if (st != DSA_OK) return st;
+  if (!indexer_ptrs_ok(q_I, q_scale, w, k_I, k_scale) || idx == nullptr) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > s->T) return DSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
+  WsLayout L = ws_layout(s, c.num_sms);
+  if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  for (int q0 = q_begin; q0 < q_begin + q_count; q0 += L.q_rows) {
+    const int cnt = (q_begin + q_count - q0) < L.q_rows ? (q_begin + q_count - q0) : L.q_rows;
+    if ((st = run_select(c, s, L, ws, q_I, q_scale, w, k_I, k_scale, q0, cnt, idx)) != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
 dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                            const int32_t* idx, uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
   dsa_status st = check_shape(s);
@@ -330,10 +464,8 @@ dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, 
     return st;
   for (int q0 = d_rows; q0 < s->T; q0 += L.q_rows) {
     const int cnt = (s->T - q0) < L.q_rows ? (s->T - q0) : L.q_rows;
-    if ((st = run_indexer(c, s, in->q_I, in->q_scale, in->w, in->k_I, in->k_scale, q0, cnt, scores, ld)) != DSA_OK)
-      return st;
-    if ((st = run_topk(c, s, scores, ld, q0, cnt, idx_out,
-                       L.topk_bytes ? static_cast<char*>(ws) + L.topk_off : nullptr, L.topk_bytes)) != DSA_OK)
+    if ((st = run_select(c, s, L, ws, in->q_I, in->q_scale, in->w, in->k_I, in->k_scale, q0, cnt, idx_out)) !=
+        DSA_OK)
       return st;
   }
   return run_attn(c, s, in->q, in->kv, in->v, idx_out, d_rows, out, lse, part, L.nsplit);

@@ -62,6 +62,13 @@ struct IdxParams {
   KvMap kv;            // per-sequence lengths, paged or contiguous key cache
   long long pool_rows; // rows of the k_I / k_scale pools
   int box_rows;        // key rows per TMA load (a key tile takes kBM / box_rows)
+  int kstride;         // column s of a score row is key s * kstride (1: every key)
+  const unsigned int* thr;   // candidate mode: per launch row, the smallest order key kept
+  unsigned int* cand_key;
+  int32_t* cand_idx;
+  unsigned int* cand_cnt;
+  int cand_cap;
+  const int* row_slot;       // repair mode: score row of each launch row (-1: skip)
   const float* w;
   const float* q_scale;
   const float* k_scale;
@@ -83,7 +90,9 @@ struct Layout {
   static constexpr int kAOff = kBOff + kMaxNB * kBSubBytes;
   static constexpr int kWOff = kAOff + kStages * kABytes;            // wM, two item buffers
   static constexpr int kWFloats = kMaxNB * kNSub;
-  static constexpr int kBarOff = kWOff + 2 * kWFloats * 4;
+  static constexpr int kThrOff = kWOff + 2 * kWFloats * 4;           // thresholds, two item buffers
+  static constexpr int kThrWords = kMaxNB * kNSub / 4;               // queries per item at most (4 heads)
+  static constexpr int kBarOff = kThrOff + 2 * kThrWords * 4;
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNAcc + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
@@ -117,8 +126,14 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
     it.t0 = p.q_begin + g * per_group;
     it.tend = min(it.t0 + per_group, q_end);
     const int pos_last = it.off + it.tend - 1;
-    it.ntiles = pos_last / kBM + 1;
+    it.ntiles = pos_last / p.kstride / kBM + 1;
     const int nch = (it.ntiles + p.kc - 1) / p.kc;
+    if (p.row_slot != nullptr) {
+      // repair mode: only query groups holding a listed row are scored
+      bool any = false;
+      for (int t = it.t0; t < it.tend && !any; ++t) any = p.row_slot[(size_t)b * p.q_count + (t - p.q_begin)] >= 0;
+      if (!any) continue;
+    }
     int c0 = (int)(((long long)cta - flat) % grid);
     if (c0 < 0) c0 += grid;
     for (int c = c0; c < nch; c += grid) {
@@ -142,8 +157,8 @@ __device__ __forceinline__ int item_nsub(const IdxParams& p, const Item& it) {
 template <int HI>
 __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, int kt, int nsub) {
   constexpr int QPS = kNSub / HI;
-  // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM - off
-  const int x = kt * kBM - it.off - it.t0 + QPS;
+  // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM * kstride - off
+  const int x = kt * kBM * p.kstride - it.off - it.t0 + QPS;
   const int j = x > 0 ? x / QPS - 1 : 0;
   return j < 0 ? 0 : (j < nsub - 1 ? j : nsub - 1);
 }
@@ -159,6 +174,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   uint8_t* sB = smem + L::kBOff;
   uint8_t* sA = smem + L::kAOff;
   float* sW = reinterpret_cast<float*>(smem + L::kWOff);
+  unsigned int* sThr = reinterpret_cast<unsigned int*>(smem + L::kThrOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + kStages;
@@ -245,8 +261,9 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           // the cache is contiguous); a run at or past L_b, or on an unmapped
           // page, reads the fill value from past the end of the pool
           for (int r0 = 0; r0 < kBM; r0 += p.box_rows) {
-            const int s = kt * kBM + r0;
-            long long y = s < it.L ? p.kv.row(it.b, s) : -1;
+            const int s = (kt * kBM + r0) * p.kstride;
+            // a key sample is a contiguous cache read every kstride-th row
+            long long y = s < it.L ? p.kv.row(it.b, s) / p.kstride : -1;
             if (y < 0) {
               if (s < it.L) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (2u << 8));
               y = p.pool_rows;
@@ -354,8 +371,16 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
         }
         wbuf[x] = v;
       }
+      if (p.thr != nullptr) {
+        unsigned int* tbuf = sThr + (items & 1) * L::kThrWords;
+        for (int x = etid; x < p.nb * QPS; x += E::EPI_THREADS) {
+          const int t = it.t0 + x;
+          tbuf[x] = t < it.tend ? p.thr[(size_t)it.b * p.q_count + (t - p.q_begin)] : 0xFFFFFFFFu;
+        }
+      }
       mbar_arrive(&w_ready[items & 1]);
       if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.wait_ns, ab)) { fail(7); return false; }
+      const unsigned int* tq = sThr + (items & 1) * L::kThrWords;
       ++items;
       const int nsub = item_nsub<HI>(p, it);
       const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
@@ -367,7 +392,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
         for (int g = 0; g < E::G; ++g) {
           sg[g] = (kt + g) * kBM + r;
           // 1/2: the head sum below accumulates 2 ReLU(x)
-          const long long kr = (g < ng && sg[g] < it.L) ? p.kv.row(it.b, sg[g]) : -1;
+          const long long kr = (g < ng && sg[g] * p.kstride < it.L) ? p.kv.row(it.b, sg[g] * p.kstride) : -1;
           ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
         }
         const int jlo = first_active<HI>(p, it, kt, nsub);
@@ -447,13 +472,42 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
 #pragma unroll
               for (int i = 0; i < NP; ++i) a += part[g][q][i].x + part[g][q][i].y;
               const int t = it.t0 + j * QPS + q;
-              if (t < it.tend && s <= it.off + t) {
-                // self-check: the score slot lies inside this launch's tile
-                const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
-                if (ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld)
-                  p.scores[ri * p.ld + s] = a * ksg[g];
-                else
-                  report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
+              const bool vis = t < it.tend && s * p.kstride <= it.off + t;
+              const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
+              if (p.thr == nullptr) {
+                if (vis) {
+                  // self-check: the score slot lies inside this launch's tile
+                  const bool in_tile = ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld;
+                  const long long so = !in_tile ? -1 : (p.row_slot != nullptr ? p.row_slot[ri] : ri);
+                  if (so >= 0)
+                    p.scores[so * p.ld + s] = a * ksg[g];
+                  else if (!in_tile)
+                    report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
+                }
+              } else {
+                // candidate mode: append the scores at or above the row's
+                // threshold, one atomic per warp and query (the warp's 32
+                // lanes hold 32 consecutive keys of the same query)
+                const unsigned int key = order_key(a * ksg[g]);
+                const bool take = vis && key >= tq[j * QPS + q];
+                const unsigned int m = __ballot_sync(0xffffffffu, take);
+                if (m != 0u) {
+                  const int leader = __ffs(m) - 1;
+                  unsigned int base = 0;
+                  if (lane == leader) base = atomicAdd(&p.cand_cnt[ri], (unsigned int)__popc(m));
+                  base = __shfl_sync(0xffffffffu, base, leader);
+                  if (take) {
+                    const unsigned int o = base + (unsigned int)__popc(m & ((1u << lane) - 1u));
+                    if (ri >= 0 && ri < (long long)p.B * p.q_count) {
+                      if (o < (unsigned int)p.cand_cap) {
+                        p.cand_key[ri * p.cand_cap + o] = key;
+                        p.cand_idx[ri * p.cand_cap + o] = s * p.kstride;
+                      }
+                    } else {
+                      report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (3u << 8));
+                    }
+                  }
+                }
               }
             }
           }
@@ -486,7 +540,12 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
     while (a.kv.page_size % box_rows != 0) box_rows >>= 1;
   const long long pool_rows = a.kv.pool_rows(a.B);
   if (box_rows < 16 || pool_rows <= 0 || pool_rows >= (1LL << 31)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.k_I, (uint64_t)pool_rows, DI, DI, box_rows, DI, sw))
+  // a key sample (kstride > 1) reads every kstride-th row of a contiguous
+  // cache: a tensor map whose row pitch is kstride rows
+  const int ks = a.kstride > 1 ? a.kstride : 1;
+  if (ks > 1 && (a.kv.page_size != 0 || a.S % ks != 0)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.k_I, (uint64_t)(pool_rows / ks), DI,
+                    (uint64_t)DI * ks, box_rows, DI, sw))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_I, (uint64_t)a.B * a.T * HI, DI, DI, kNSub, DI, sw))
     return cudaErrorInvalidValue;
@@ -494,6 +553,13 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   p.kv = a.kv;
   p.pool_rows = pool_rows;
   p.box_rows = box_rows;
+  p.kstride = ks;
+  p.thr = a.thr;
+  p.cand_key = a.cand_key;
+  p.cand_idx = a.cand_idx;
+  p.cand_cnt = a.cand_cnt;
+  p.cand_cap = a.cand_cap;
+  p.row_slot = a.row_slot;
   p.w = a.w;
   p.q_scale = a.q_scale;
   p.k_scale = a.k_scale;
@@ -517,7 +583,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
     for (int g = 0; g < p.groups_per_seq; ++g) {
       const int t0 = a.q_begin + g * per_group;
       const int tend = t0 + per_group < a.q_begin + a.q_count ? t0 + per_group : a.q_begin + a.q_count;
-      const int ntiles = (a.S - a.T + tend - 1) / kBM + 1;
+      const int ntiles = (a.S - a.T + tend - 1) / ks / kBM + 1;
       n += (ntiles + kc - 1) / kc;
     }
     return n * a.B;

@@ -28,6 +28,14 @@ enum : unsigned int {
 __device__ __forceinline__ void report_error(DevErr* e, unsigned int code, unsigned int detail) {
   if (e != nullptr && atomicCAS(&e->code, 0u, code) == 0u) atomicExch(&e->detail, detail);
 }
+
+// Order-preserving 32-bit key of a score: a > b as floats iff key(a) >
+// key(b) as unsigned integers; -0.0 is folded onto +0.0.
+__device__ __forceinline__ unsigned int order_key(float f) {
+  unsigned int u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 #endif
 
 // Where the keys of each sequence are: per-sequence lengths and the
@@ -79,6 +87,18 @@ struct LaunchCtx {
 
 struct IndexerArgs {
   KvMap kv;
+  int kstride;              // score every kstride-th key only (a sample; contiguous caches, S % kstride == 0)
+  // candidate mode (thr set): instead of writing score rows, append the
+  // (order key, key index) of every visible score whose key is >= thr[row]
+  // to row's list of cand_cap slots, counting in cand_cnt[row]
+  const unsigned int* thr;
+  unsigned int* cand_key;
+  int32_t* cand_idx;
+  unsigned int* cand_cnt;
+  int cand_cap;
+  // repair mode (row_slot set): score only the rows with row_slot[row] >= 0,
+  // into score row row_slot[row]; work items without such a row are skipped
+  const int* row_slot;
   const uint8_t* q_I;
   const float* q_scale;
   const float* w;
@@ -132,6 +152,18 @@ cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a);
 cudaError_t launch_topk_merge(const LaunchCtx& c, const float* cand_scores, const int32_t* cand_idx, int rows,
                               int nparts, int k, int32_t* idx, int local_begin, int local_count, int32_t* idx_local);
 int topk_merge_max_candidates();
+
+// selection without a score tile (topk.cu; the indexer's sample and
+// candidate modes feed it)
+int topk_cand_cap();
+cudaError_t launch_topk_threshold(const LaunchCtx& c, const TopkArgs& a, const float* sample, long long ld_s,
+                                  int kstride, int target, unsigned int* thr, unsigned int* cnt, int* row_slot,
+                                  unsigned int* nfail);
+cudaError_t launch_topk_cand_select(const LaunchCtx& c, const TopkArgs& a, const unsigned int* cand_key,
+                                    const int32_t* cand_idx, const unsigned int* cnt, int cap, int* row_slot,
+                                    int* fail_rows, unsigned int* nfail, int max_fail);
+cudaError_t launch_topk_repair(const LaunchCtx& c, const TopkArgs& a, const float* tile, long long ld,
+                               const int* fail_rows, const unsigned int* nfail, int max_fail);
 
 cudaError_t launch_wait_timeout_probe(const LaunchCtx& c);
 

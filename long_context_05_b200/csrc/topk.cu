@@ -51,12 +51,6 @@ constexpr int kWsKeys = kBins + 4;
 constexpr int kWsIdx = kWsKeys + kCap;
 constexpr int kWsRowWords = kWsIdx + kCap;
 
-__device__ __forceinline__ unsigned int order_key(float f) {
-  unsigned int u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Block-wide inclusive scan of one value per thread; returns the inclusive
 // prefix and writes the block total to *total.
 __device__ __forceinline__ unsigned int block_scan(unsigned int v, unsigned int* warp_tot, unsigned int* total) {
@@ -432,19 +426,8 @@ __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& 
   return true;
 }
 
-// One block per row.
-__global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevErr* err) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  int b, t, n;
-  const float* row;
-  int32_t* out;
-  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
-  const int k = a.k;
-  if (n <= k) {
-    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
-    return;
-  }
+// The whole selection of one row held in memory (n > k visible scores).
+__device__ void select_row(const float* row, int n, int k, int32_t* out, Smem& sm, DevErr* err) {
   if (single_pass(row, n, k, out, sm, err)) return;
   // two passes: histogram of the top 11 bits, then the threshold bin
   __syncthreads();
@@ -458,6 +441,134 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevEr
   const unsigned int inbin = B < (unsigned)kBins ? sm.hist[B] : 0u;
   __syncthreads();
   select_from_bin(row, n, k, out, B, above, inbin, sm, err);
+}
+
+// One block per row.
+__global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
+  const int k = a.k;
+  if (n <= k) {
+    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
+    return;
+  }
+  select_row(row, n, k, out, sm, err);
+}
+
+// ---------------------------------------------------------------- selection without a score tile
+// The indexer first scores a strided sample of the keys (column j = key
+// j * kstride) into a small tile; per row, the rank-rs sample score is a
+// threshold at or above which about `target` keys of the whole row are
+// expected.  The indexer then scores every key and appends the (order key,
+// index) pairs at or above the row's threshold to the row's candidate list
+// (at most cap slots), and one block per row selects among them exactly:
+// every key at or above the threshold is a candidate, so with at least k
+// candidates and no overflow the row's top k are among them.  Rows whose
+// candidates fall short or overflow are listed for repair: the indexer scores
+// just those rows into a small tile and select_row finishes them.
+
+// Threshold per row, its candidate count cleared, its repair slot unset.
+__global__ void __launch_bounds__(kThreads, 2)
+    topk_threshold_kernel(TopkArgs a, const float* sample, long long ld_s, int kstride, int target,
+                          unsigned int* thr, unsigned int* cnt, int* row_slot, unsigned int* nfail, DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int r = blockIdx.x;
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, r, err, &b, &t, &n, &row, &out);
+  if (threadIdx.x == 0) {
+    cnt[r] = 0u;
+    row_slot[r] = -1;
+    if (r == 0) *nfail = 0u;
+  }
+  if (n <= kCap) {  // the candidate list holds every visible key
+    if (threadIdx.x == 0) thr[r] = 0u;
+    return;
+  }
+  const int ns = (n - 1) / kstride + 1;          // visible sample keys
+  long long rs = ((long long)target * ns + n - 1) / n;
+  if (rs < 1) rs = 1;
+  if (rs > ns) rs = ns;
+  const float* srow = sample + (size_t)r * ld_s;
+  unsigned int krem, key;
+  if (ns <= kCap) {
+    for (int i = threadIdx.x; i < ns; i += kThreads) sm.ck[i] = order_key(srow[i]);
+    __syncthreads();
+    const unsigned int* ck = sm.ck;
+    key = radix_select([ck](int i) { return ck[i]; }, ns, 0u, 0u, 32, (unsigned int)rs, sm.hist, sm.warp_tot,
+                       &sm.bin, &sm.above, &sm.total, &krem);
+  } else {
+    key = radix_select([srow](int i) { return order_key(srow[i]); }, ns, 0u, 0u, 32, (unsigned int)rs, sm.hist,
+                       sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
+  }
+  if (threadIdx.x == 0) thr[r] = key;
+}
+
+// Exact selection among a row's candidates; a row that cannot be finished
+// from them is listed for repair (and gets the best selection its candidates
+// allow in the meantime).
+__global__ void __launch_bounds__(kThreads, 2)
+    topk_cand_select_kernel(TopkArgs a, const unsigned int* cand_key, const int32_t* cand_idx,
+                            const unsigned int* cnt, int cap, int* row_slot, int* fail_rows, unsigned int* nfail,
+                            int max_fail, DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int r = blockIdx.x;
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, r, err, &b, &t, &n, &row, &out);
+  const int k = a.k;
+  if (n <= k) {
+    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
+    return;
+  }
+  const unsigned int c = cnt[r];
+  const bool complete = c >= (unsigned int)k && c <= (unsigned int)cap && c <= (unsigned int)kCap;
+  const int nc = (int)min(c, (unsigned int)min(cap, kCap));
+  for (int i = threadIdx.x; i < nc; i += kThreads) {
+    sm.ck[i] = cand_key[(size_t)r * cap + i];
+    sm.ci[i] = cand_idx[(size_t)r * cap + i];
+  }
+  if (threadIdx.x == 0) sm.cnt = 0;
+  __syncthreads();
+  const int keep = min(nc, k);
+  if (keep > 0) select_candidates(nc, 0u, 0u, 32, (unsigned int)keep, k, out, sm, err);
+  __syncthreads();
+  for (int x = keep + threadIdx.x; x < k; x += kThreads) out[x] = -1;
+  if (!complete && threadIdx.x == 0) {
+    const unsigned int slot = atomicAdd(nfail, 1u);
+    if (slot < (unsigned int)max_fail) {
+      fail_rows[slot] = r;
+      row_slot[r] = (int)slot;
+    } else {
+      report_error(err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_TOPK | (0x40u << 8));
+    }
+  }
+}
+
+// Repair: rows listed by topk_cand_select_kernel, scored in full into
+// tile[slot] by the indexer, selected as topk_row_kernel would.
+__global__ void __launch_bounds__(kThreads, 2)
+    topk_repair_kernel(TopkArgs a, const float* tile, long long ld, const int* fail_rows, const unsigned int* nfail,
+                       int max_fail, DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int slot = blockIdx.x;
+  if ((unsigned int)slot >= min(*nfail, (unsigned int)max_fail)) return;
+  const int r = fail_rows[slot];
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, r, err, &b, &t, &n, &row, &out);
+  if (n <= a.k) return;  // never listed
+  select_row(tile + (size_t)slot * ld, n, a.k, out, sm, err);
 }
 
 // ---------------------------------------------------------------- split path
@@ -762,6 +873,46 @@ cudaError_t launch_topk_merge(const LaunchCtx& c, const float* cand_scores, cons
 }
 
 int topk_merge_max_candidates() { return kCap; }
+
+int topk_cand_cap() { return kCap; }
+
+cudaError_t launch_topk_threshold(const LaunchCtx& c, const TopkArgs& a, const float* sample, long long ld_s,
+                                  int kstride, int target, unsigned int* thr, unsigned int* cnt, int* row_slot,
+                                  unsigned int* nfail) {
+  const int rows = a.B * a.q_count;
+  if (rows <= 0) return cudaSuccess;
+  const size_t smem = sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_threshold_kernel<<<rows, kThreads, smem, c.stream>>>(a, sample, ld_s, kstride, target, thr, cnt, row_slot,
+                                                            nfail, c.err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_cand_select(const LaunchCtx& c, const TopkArgs& a, const unsigned int* cand_key,
+                                    const int32_t* cand_idx, const unsigned int* cnt, int cap, int* row_slot,
+                                    int* fail_rows, unsigned int* nfail, int max_fail) {
+  const int rows = a.B * a.q_count;
+  if (rows <= 0) return cudaSuccess;
+  const size_t smem = sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_cand_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_cand_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, cand_key, cand_idx, cnt, cap, row_slot, fail_rows,
+                                                              nfail, max_fail, c.err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_repair(const LaunchCtx& c, const TopkArgs& a, const float* tile, long long ld,
+                               const int* fail_rows, const unsigned int* nfail, int max_fail) {
+  const size_t smem = sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_repair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_repair_kernel<<<max_fail, kThreads, smem, c.stream>>>(a, tile, ld, fail_rows, nfail, max_fail, c.err);
+  note_launches(1);
+  return cudaGetLastError();
+}
 
 // Split path with a caller-provided histogram array (B * q_count * 2048
 // words): zero it, histogram each row over several blocks, select per row.

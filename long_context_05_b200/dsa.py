@@ -28,7 +28,8 @@ EXPORTS = [
     "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk",
     "dsa_sparse_attn", "dsa_forward", "dsa_prefill", "dsa_decode", "dsa_get_device_error",
     "dsa_set_wait_timeout_us", "dsa_launch_count", "dsa_selftest_wait_timeout", "dsa_topk_static",
-    "dsa_dense_attn", "dsa_topk_candidates", "dsa_topk_merge", "dsa_attn_combine",
+    "dsa_dense_attn", "dsa_topk_candidates", "dsa_topk_merge", "dsa_attn_combine", "dsa_select",
+    "dsa_kl_target", "dsa_indexer_kl", "dsa_indexer_backward",
 ]
 
 
@@ -82,6 +83,14 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_attn.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.dsa_dense_attn.restype = i
         L.dsa_dense_attn.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_kl_target.restype = i
+        L.dsa_kl_target.argtypes = [sp, vp, vp, vp, vp, i, i, vp, i64, vp]
+        L.dsa_indexer_kl.restype = i
+        L.dsa_indexer_kl.argtypes = [sp, vp, vp, i64, vp, i, i, vp, vp, vp]
+        L.dsa_indexer_backward.restype = i
+        L.dsa_indexer_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, i64, vp, i, i, vp, vp, vp, vp]
+        L.dsa_select.restype = i
+        L.dsa_select.argtypes = [sp, vp, vp, vp, vp, vp, i, i, vp, vp, sz, vp]
         L.dsa_topk_candidates.restype = i
         L.dsa_topk_candidates.argtypes = [sp, vp, i64, vp, ctypes.c_int32, vp, vp, vp]
         L.dsa_topk_merge.restype = i
@@ -194,6 +203,18 @@ def topk(shape: Shape, scores: torch.Tensor, q_begin: int, q_count: int, idx: to
     return idx
 
 
+def select(shape: Shape, q_I, q_scale, w, k_I, k_scale, q_begin: int, q_count: int, idx: torch.Tensor,
+           ws: torch.Tensor) -> torch.Tensor:
+    """Steps A and B for queries [q_begin, q_begin + q_count) -> idx [B, T, k]."""
+    for t, d, n in ((q_I, torch.uint8, "q_I"), (q_scale, torch.float32, "q_scale"), (w, torch.float32, "w"),
+                    (k_I, torch.uint8, "k_I"), (k_scale, torch.float32, "k_scale"), (idx, torch.int32, "idx")):
+        _need(t, d, n)
+    _check("dsa_select", lib().dsa_select(
+        ctypes.byref(shape), _p(q_I), _p(q_scale), _p(w), _p(k_I), _p(k_scale), q_begin, q_count, _p(idx),
+        _p(ws), ws.numel(), _stream()))
+    return idx
+
+
 def topk_static(shape: Shape, scores: torch.Tensor, q_begin: int, q_count: int,
                 idx: torch.Tensor) -> torch.Tensor:
     """Step B with the library's fixed histogram array (no workspace, no allocation)."""
@@ -272,6 +293,47 @@ def attn_combine(shape: Shape, o_parts, lse_parts, out, lse=None):
     _check("dsa_attn_combine", lib().dsa_attn_combine(
         ctypes.byref(shape), o_parts.shape[0], _p(o_parts), _p(lse_parts), _p(out), _p(lse), _stream()))
     return out, lse
+
+
+def kl_target(shape: Shape, q, kv, lse, q_begin: int, q_count: int, target, idx=None):
+    """Indexer-training target rows [B * q_count, ld] from the main attention's lse."""
+    _need(q, torch.bfloat16, "q")
+    _need(kv, torch.bfloat16, "kv")
+    _need(lse, torch.float32, "lse")
+    _need(target, torch.float32, "target")
+    if idx is not None:
+        _need(idx, torch.int32, "idx")
+    _check("dsa_kl_target", lib().dsa_kl_target(
+        ctypes.byref(shape), _p(q), _p(kv), _p(lse), _p(idx), q_begin, q_count, _p(target), target.shape[-1],
+        _stream()))
+    return target
+
+
+def indexer_kl(shape: Shape, scores, target, q_begin: int, q_count: int, grad, loss, idx=None):
+    """KL loss per row and its gradient with respect to the indexer scores."""
+    for t, n in ((scores, "scores"), (target, "target"), (grad, "grad"), (loss, "loss")):
+        _need(t, torch.float32, n)
+    if idx is not None:
+        _need(idx, torch.int32, "idx")
+    _check("dsa_indexer_kl", lib().dsa_indexer_kl(
+        ctypes.byref(shape), _p(scores), _p(target), scores.shape[-1], _p(idx), q_begin, q_count, _p(grad),
+        _p(loss), _stream()))
+    return grad, loss
+
+
+def indexer_backward(shape: Shape, q_I, q_scale, w, k_I, k_scale, grad, q_begin: int, q_count: int, dq, dw, dk,
+                     idx=None):
+    """Gradients of the indexer's inputs (dequantised, FP32); dk accumulates."""
+    for t, d, n in ((q_I, torch.uint8, "q_I"), (q_scale, torch.float32, "q_scale"), (w, torch.float32, "w"),
+                    (k_I, torch.uint8, "k_I"), (k_scale, torch.float32, "k_scale"), (grad, torch.float32, "grad"),
+                    (dq, torch.float32, "dq"), (dw, torch.float32, "dw"), (dk, torch.float32, "dk")):
+        _need(t, d, n)
+    if idx is not None:
+        _need(idx, torch.int32, "idx")
+    _check("dsa_indexer_backward", lib().dsa_indexer_backward(
+        ctypes.byref(shape), _p(q_I), _p(q_scale), _p(w), _p(k_I), _p(k_scale), _p(grad), grad.shape[-1], _p(idx),
+        q_begin, q_count, _p(dq), _p(dw), _p(dk), _stream()))
+    return dq, dw, dk
 
 
 def _inputs(inp: dict) -> Inputs:

@@ -260,6 +260,75 @@ def combine_partials(o_parts, lse_parts):
 
 
 # ---------------------------------------------------------------------------
+# training the indexer (kernel level)
+# ---------------------------------------------------------------------------
+#
+# tenelement.pl, "DeepSeek V3.2-Exp Cuts Long-Context Costs ...", section
+# "Proces Treningu DSA: Od Warm-up do Sparsity": in a short warm-up the
+# indexer learns the dense model's attention distribution through a KL
+# divergence while the main model is frozen; then a sparse stage trains with
+# top-k = 2048, and the indexer's gradients stay separate from the main
+# language loss (ouchyi thread, "Nasil calisiyor": the indexer is aligned by
+# KL divergence first).  Readings where the pages are silent: the target of
+# query t is the main attention's weights summed over heads and divided by H
+# (an L1-normalised distribution over keys); the loss is KL(target ||
+# softmax(I[t, .])) over the visible keys (warm-up) or over the selected set
+# (sparse stage, where both distributions are taken over the set); the target
+# is a constant (no gradient flows into the main attention).
+
+
+def kl_target_row(q_t, kv, pos: int, tau: float, sel=None) -> np.ndarray:
+    """Target distribution of query t: p[s] = (1/H) sum_h softmax_s(tau q_h . kv[s])
+    over the visible keys 0..pos, or over the selected set `sel` (-1 = empty
+    slot) when given.  Returns float64 [pos + 1] (zero outside the set)."""
+    keys = np.arange(pos + 1) if sel is None else np.unique(np.asarray(sel)[np.asarray(sel) >= 0])
+    K = np.asarray(kv[keys], np.float64)
+    z = tau * (np.asarray(q_t, np.float64) @ K.T)               # [H, n]
+    z = z - z.max(axis=1, keepdims=True)
+    a = np.exp(z)
+    a = a / a.sum(axis=1, keepdims=True)
+    p = np.zeros(pos + 1)
+    p[keys] = a.mean(axis=0)
+    return p
+
+
+def indexer_kl_row(scores_t, p_t, sel=None):
+    """KL(p || softmax(I)) of one query row and its gradient with respect to
+    the scores.  scores_t, p_t: float64 [n] over keys 0..pos; with `sel`, both
+    distributions are over the selected set only.  With q = softmax(I) over
+    the set, loss = sum_s p_s (ln p_s - ln q_s) (terms with p_s = 0 are 0) and
+    dloss/dI_s = q_s - p_s (zero outside the set).  Returns (loss, grad [n])."""
+    I = np.asarray(scores_t, np.float64)
+    n = I.shape[0]
+    keys = np.arange(n) if sel is None else np.unique(np.asarray(sel)[np.asarray(sel) >= 0])
+    z = I[keys] - I[keys].max()
+    lq = z - np.log(np.exp(z).sum())
+    ps = np.asarray(p_t, np.float64)[keys]
+    nz = ps > 0
+    loss = float(np.sum(ps[nz] * (np.log(ps[nz]) - lq[nz])))
+    g = np.zeros(n)
+    g[keys] = np.exp(lq) - ps
+    return loss, g
+
+
+def indexer_grads_row(qd_t, w_t, kd, pos: int, g_t):
+    """Chain rule of sum_s g_s I[t, s] back to the indexer's inputs, with
+    I[t, s] = sum_j w_j ReLU(q_j . k_s) on the dequantised operands:
+        dw_j  = sum_s g_s ReLU(q_j . k_s)
+        dq_j  = sum_s g_s w_j [q_j . k_s > 0] k_s
+        dk_s  = sum_j g_s w_j [q_j . k_s > 0] q_j      (row t's contribution)
+    g_t: float64 [pos + 1].  Returns (dq [H_I, D_I], dw [H_I], dk [pos + 1, D_I])."""
+    Q = np.asarray(qd_t, np.float64)
+    K = np.asarray(kd[: pos + 1], np.float64)
+    w = np.asarray(w_t, np.float64)
+    g = np.asarray(g_t, np.float64)
+    dots = Q @ K.T                                              # [H_I, n]
+    dw = np.maximum(dots, 0.0) @ g
+    G = (w[:, None] * (dots > 0)) * g[None, :]                  # [H_I, n]
+    return G @ K, dw, G.T @ Q
+
+
+# ---------------------------------------------------------------------------
 # the whole path, and the work it touches
 # ---------------------------------------------------------------------------
 

@@ -362,3 +362,79 @@ def test_work_counts_o_lk():
     a2 = O.work_counts(8192, 8192, 2048)["attention_pairs"]
     assert a2 - a1 == 4096 * 2048           # linear in L beyond k
     assert O.work_counts(1, 131072, 2048)["attention_pairs"] == 2048
+
+
+# ---------------------------------------------------------------- indexer training
+
+def _train_case(seed=21, HI=3, DI=5, S=12, H=4, dk=6):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((HI, DI)), rng.standard_normal(HI), rng.standard_normal((S, DI)),
+            rng.standard_normal((H, dk)), rng.standard_normal((S, dk)))
+
+
+def test_kl_target_is_head_mean_of_dense_attention_weights():
+    """p sums to 1 and p @ V equals the mean over heads of the independent
+    dense attention output (the target is the heads' weights averaged)."""
+    _, _, _, q, kv = _train_case()
+    pos, tau, dv = 9, 0.4, 3
+    p = O.kl_target_row(q, kv, pos, tau)
+    assert abs(p.sum() - 1.0) < 1e-14 and np.all(p >= 0)
+    o, _ = O.dense_causal_attention_row(q, kv, pos, dv, tau)
+    assert np.allclose(p @ kv[: pos + 1, :dv], o.mean(0), atol=1e-14)
+    # over a selected set: zero outside it, and the same identity with the
+    # sparse attention
+    sel = np.array([7, 2, -1, 5, 9])
+    ps = O.kl_target_row(q, kv, pos, tau, sel)
+    assert np.all(ps[[0, 1, 3, 4, 6, 8]] == 0) and abs(ps.sum() - 1) < 1e-14
+    os_, _ = O.sparse_attention_row(q, kv, sel, dv, tau)
+    assert np.allclose(ps @ kv[: pos + 1, :dv], os_.mean(0), atol=1e-14)
+
+
+def test_indexer_kl_loss_and_score_gradient():
+    rng = np.random.default_rng(22)
+    I = rng.standard_normal(10)
+    p = rng.random(10)
+    p /= p.sum()
+    loss, g = O.indexer_kl_row(I, p)
+    assert loss >= 0
+    q = np.exp(I - I.max()); q /= q.sum()
+    assert abs(loss - np.sum(p * np.log(p / q))) < 1e-13
+    # gradient by central differences
+    for s in range(10):
+        e = np.zeros(10); e[s] = 1e-6
+        fd = (O.indexer_kl_row(I + e, p)[0] - O.indexer_kl_row(I - e, p)[0]) / 2e-6
+        assert abs(fd - g[s]) < 1e-8
+    # p == softmax(I): no loss, no gradient
+    l0, g0 = O.indexer_kl_row(I, q)
+    assert abs(l0) < 1e-14 and np.max(np.abs(g0)) < 1e-15
+    # over a set: the other keys get no gradient
+    sel = np.array([1, 4, 6])
+    pset = np.zeros(10); pset[sel] = p[sel] / p[sel].sum()      # a target over the set
+    ls, gs = O.indexer_kl_row(I, pset, sel)
+    assert np.all(gs[[0, 2, 3, 5, 7, 8, 9]] == 0) and abs(gs.sum()) < 1e-14
+
+
+def test_indexer_input_gradients_by_finite_differences():
+    """dq, dw, dk of the KL loss through the indexer, against central
+    differences of the loss as a function of the inputs."""
+    Q, w, K, q, kv = _train_case()
+    pos, tau = 10, 0.5
+    p = O.kl_target_row(q, kv, pos, tau)
+
+    def loss(Q_, w_, K_):
+        return O.indexer_kl_row(O.indexer_row(Q_, w_, K_, pos), p)[0]
+
+    _, g = O.indexer_kl_row(O.indexer_row(Q, w, K, pos), p)
+    dq, dw, dk = O.indexer_grads_row(Q, w, K, pos, g)
+    h = 1e-6
+    for (j, d) in [(0, 0), (1, 3), (2, 4)]:
+        E = np.zeros_like(Q); E[j, d] = h
+        assert abs((loss(Q + E, w, K) - loss(Q - E, w, K)) / (2 * h) - dq[j, d]) < 1e-7
+    for j in range(3):
+        e = np.zeros(3); e[j] = h
+        assert abs((loss(Q, w + e, K) - loss(Q, w - e, K)) / (2 * h) - dw[j]) < 1e-7
+    for (s_, d) in [(0, 1), (5, 2), (10, 4)]:
+        E = np.zeros_like(K); E[s_, d] = h
+        assert abs((loss(Q, w, K + E) - loss(Q, w, K - E)) / (2 * h) - dk[s_, d]) < 1e-7
+    # keys past pos play no part
+    assert dk.shape[0] == pos + 1
