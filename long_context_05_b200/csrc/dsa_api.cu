@@ -215,7 +215,7 @@ dsa_status run_indexer(const LaunchCtx& c, const dsa_shape* s, const uint8_t* q_
 
 dsa_status run_topk(const LaunchCtx& c, const dsa_shape* s, const float* scores, int64_t ld, int q_begin,
                     int q_count, int32_t* idx, void* ws, size_t ws_bytes) {
-  TopkArgs a;
+  TopkArgs a = {};
   a.kv = kv_map(s);
   a.scores = scores; a.ld = ld; a.idx = idx;
   a.B = s->B; a.T = s->T; a.S = s->S; a.k = s->k;
@@ -244,7 +244,7 @@ dsa_status run_select_fused(const LaunchCtx& c, const dsa_shape* s, const WsLayo
   ia.q_I = q_I; ia.q_scale = q_scale; ia.w = w; ia.k_I = k_I; ia.k_scale = k_scale;
   ia.B = s->B; ia.T = s->T; ia.S = s->S; ia.H_I = s->H_I; ia.D_I = s->D_I;
   ia.q_begin = q0; ia.q_count = cnt;
-  TopkArgs ta;
+  TopkArgs ta = {};
   ta.kv = kv_map(s);
   ta.scores = nullptr; ta.ld = 0; ta.idx = idx;
   ta.B = s->B; ta.T = s->T; ta.S = s->S; ta.k = s->k;
@@ -306,7 +306,7 @@ dsa_status run_select(const LaunchCtx& c, const dsa_shape* s, const WsLayout& L,
 dsa_status run_attn(const LaunchCtx& c, const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
                     const uint16_t* v, const int32_t* idx, int dense_rows, uint16_t* out, float* lse, float* part,
                     int nsplit) {
-  AttnArgs a;
+  AttnArgs a = {};
   a.map = kv_map(s);
   a.q = q; a.kv = kv; a.v = v; a.idx = idx; a.dense_rows = dense_rows;
   a.out = out; a.lse = lse; a.part = part;
@@ -326,6 +326,7 @@ bool indexer_ptrs_ok(const uint8_t* q_I, const float* q_scale, const float* w, c
 }  // namespace
 
 dsa_status api_check_shape(const dsa_shape* s) { return check_shape(s); }
+KvMap api_kv_map(const dsa_shape* s) { return kv_map(s); }
 dsa_status api_make_ctx(void* stream, LaunchCtx* c) { return make_ctx(stream, c); }
 
 }  // namespace dsa

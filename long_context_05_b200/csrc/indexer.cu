@@ -109,8 +109,10 @@ struct Item {
   int off;  // L - T: pos(t) = off + t
 };
 
-template <int HI, class F>
+template <int HI, bool PLAIN, class F>
 __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
+  const int KS = PLAIN ? 1 : p.kstride;
+  const int* const SLOT = PLAIN ? nullptr : p.row_slot;
   constexpr int QPS = kNSub / HI;
   const int per_group = p.nb * QPS;
   const int grid = gridDim.x, cta = blockIdx.x;
@@ -126,12 +128,12 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
     it.t0 = p.q_begin + g * per_group;
     it.tend = min(it.t0 + per_group, q_end);
     const int pos_last = it.off + it.tend - 1;
-    it.ntiles = pos_last / p.kstride / kBM + 1;
+    it.ntiles = pos_last / KS / kBM + 1;
     const int nch = (it.ntiles + p.kc - 1) / p.kc;
-    if (p.row_slot != nullptr) {
+    if (SLOT != nullptr) {
       // repair mode: only query groups holding a listed row are scored
       bool any = false;
-      for (int t = it.t0; t < it.tend && !any; ++t) any = p.row_slot[(size_t)b * p.q_count + (t - p.q_begin)] >= 0;
+      for (int t = it.t0; t < it.tend && !any; ++t) any = SLOT[(size_t)b * p.q_count + (t - p.q_begin)] >= 0;
       if (!any) continue;
     }
     int c0 = (int)(((long long)cta - flat) % grid);
@@ -154,21 +156,28 @@ __device__ __forceinline__ int item_nsub(const IdxParams& p, const Item& it) {
   constexpr int QPS = kNSub / HI;
   return min(p.nb, (it.tend - it.t0 + QPS - 1) / QPS);
 }
-template <int HI>
+template <int HI, bool PLAIN>
 __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, int kt, int nsub) {
   constexpr int QPS = kNSub / HI;
   // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM * kstride - off
-  const int x = kt * kBM * p.kstride - it.off - it.t0 + QPS;
+  const int x = kt * kBM * (PLAIN ? 1 : p.kstride) - it.off - it.t0 + QPS;
   const int j = x > 0 ? x / QPS - 1 : 0;
   return j < 0 ? 0 : (j < nsub - 1 ? j : nsub - 1);
 }
 
-template <int DI, int HI>
+// PLAIN: every key scored into score rows (stride 1, no thresholds, no repair
+// list); the general form adds the key sample, the candidate and the repair
+// modes, whose per-element checks the plain form must not pay.
+template <int DI, int HI, bool PLAIN>
 __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                       IdxParams p) {
   using L = Layout<DI>;
   constexpr int QPS = kNSub / HI;
+  // the plain form sees constants: no sample stride, no candidates, no repair
+  const int KS = PLAIN ? 1 : p.kstride;
+  const unsigned int* const THR = PLAIN ? nullptr : p.thr;
+  const int* const SLOT = PLAIN ? nullptr : p.row_slot;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem + L::kBOff;
@@ -239,7 +248,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       bool issued[kStages];
       for (int i = 0; i < kStages; ++i) issued[i] = false;
       bool ok = true;
-      for_each_item<HI>(p, [&](const Item& it) {
+      for_each_item<HI, PLAIN>(p, [&](const Item& it) {
         const int bb = nbbuf == 2 ? (int)(items & 1) : 0;
         const uint32_t use = nbbuf == 2 ? items >> 1 : items;
         if (!mbar_wait(&b_empty[bb], (use & 1) ^ 1, p.wait_ns, ab)) { fail(1); ok = false; return false; }
@@ -261,9 +270,12 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           // the cache is contiguous); a run at or past L_b, or on an unmapped
           // page, reads the fill value from past the end of the pool
           for (int r0 = 0; r0 < kBM; r0 += p.box_rows) {
-            const int s = (kt * kBM + r0) * p.kstride;
-            // a key sample is a contiguous cache read every kstride-th row
-            long long y = s < it.L ? p.kv.row(it.b, s) / p.kstride : -1;
+            const int s = (kt * kBM + r0) * KS;
+            // a key sample is a contiguous cache read every kstride-th row:
+            // row b * (S / kstride) + sample index of the strided map
+            long long y = s >= it.L ? -1
+                          : KS == 1 ? p.kv.row(it.b, s)
+                                           : (long long)it.b * (p.S / KS) + kt * kBM + r0;
             if (y < 0) {
               if (s < it.L) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (2u << 8));
               y = p.pool_rows;
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       // descriptors built once; a stage or sub-tile only adds its offset >> 4
       const uint64_t adesc0 = make_sdesc(smem_u32(sA), 16, L::kSBO, L::kSwizzleLayout);
       const uint64_t bdesc0 = make_sdesc(smem_u32(sB), 16, L::kSBO, L::kSwizzleLayout);
-      for_each_item<HI>(p, [&](const Item& it) {
+      for_each_item<HI, PLAIN>(p, [&](const Item& it) {
         const int bb = nbbuf == 2 ? (int)(items & 1) : 0;
         const uint32_t use = nbbuf == 2 ? items >> 1 : items;
         if (!mbar_wait(&b_full[bb], use & 1, p.wait_ns, ab)) { fail(3); return false; }
@@ -317,7 +329,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           tc_fence_after();
           // the first active sub-tile of kt also covers kt + 1 (later keys
           // need later queries); masked pairs are computed and dropped
-          for (int j = first_active<HI>(p, it, kt, nsub); j < nsub; ++j) {
+          for (int j = first_active<HI, PLAIN>(p, it, kt, nsub); j < nsub; ++j) {
             const int slot = u % E::NSLOT;
             if (!mbar_test_wait(&acc_empty[slot], ((u / E::NSLOT) & 1) ^ 1) &&
                 !mbar_wait(&acc_empty[slot], ((u / E::NSLOT) & 1) ^ 1, p.wait_ns, ab)) {
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     const int r = quarter * 32 + lane;   // key row within a tile
     const int etid = threadIdx.x - 64;
     uint32_t u = 0, items = 0;
-    for_each_item<HI>(p, [&](const Item& it) {
+    for_each_item<HI, PLAIN>(p, [&](const Item& it) {
       // per-item head weights  wM[(query, head)] = w * q_scale  (0 past the end)
       float* wbuf = sW + (items & 1) * L::kWFloats;
       for (int x = etid; x < p.nb * kNSub; x += E::EPI_THREADS) {
@@ -371,11 +383,11 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
         }
         wbuf[x] = v;
       }
-      if (p.thr != nullptr) {
+      if (THR != nullptr) {
         unsigned int* tbuf = sThr + (items & 1) * L::kThrWords;
         for (int x = etid; x < p.nb * QPS; x += E::EPI_THREADS) {
           const int t = it.t0 + x;
-          tbuf[x] = t < it.tend ? p.thr[(size_t)it.b * p.q_count + (t - p.q_begin)] : 0xFFFFFFFFu;
+          tbuf[x] = t < it.tend ? THR[(size_t)it.b * p.q_count + (t - p.q_begin)] : 0xFFFFFFFFu;
         }
       }
       mbar_arrive(&w_ready[items & 1]);
@@ -386,16 +398,17 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
       for (int kt = kt0; kt < kt1; kt += E::G) {
         const int ng = min(E::G, kt1 - kt);
-        int sg[E::G];
+        int sg[E::G], spos[E::G];
         float ksg[E::G];
 #pragma unroll
         for (int g = 0; g < E::G; ++g) {
           sg[g] = (kt + g) * kBM + r;
           // 1/2: the head sum below accumulates 2 ReLU(x)
-          const long long kr = (g < ng && sg[g] * p.kstride < it.L) ? p.kv.row(it.b, sg[g] * p.kstride) : -1;
+          spos[g] = sg[g] * KS;   // key position of column sg[g]
+          const long long kr = (g < ng && spos[g] < it.L) ? p.kv.row(it.b, spos[g]) : -1;
           ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
         }
-        const int jlo = first_active<HI>(p, it, kt, nsub);
+        const int jlo = first_active<HI, PLAIN>(p, it, kt, nsub);
         const uint32_t u0 = u;
         u += (uint32_t)(nsub - jlo);
         // this group's sub-tiles: my = u0 + (j - jlo) == grp (mod NGRP)
@@ -466,25 +479,27 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           for (int g = 0; g < E::G; ++g) {
             if (g >= ng) break;
             const int s = sg[g];
+            const int sp = spos[g];
 #pragma unroll
             for (int q = 0; q < QPS; ++q) {
               float a = 0.f;
 #pragma unroll
               for (int i = 0; i < NP; ++i) a += part[g][q][i].x + part[g][q][i].y;
               const int t = it.t0 + j * QPS + q;
-              const bool vis = t < it.tend && s * p.kstride <= it.off + t;
-              const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
-              if (p.thr == nullptr) {
+              const bool vis = t < it.tend && sp <= it.off + t;
+              if (THR == nullptr) {
                 if (vis) {
                   // self-check: the score slot lies inside this launch's tile
+                  const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
                   const bool in_tile = ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld;
-                  const long long so = !in_tile ? -1 : (p.row_slot != nullptr ? p.row_slot[ri] : ri);
+                  const long long so = !in_tile ? -1 : (SLOT != nullptr ? SLOT[ri] : ri);
                   if (so >= 0)
                     p.scores[so * p.ld + s] = a * ksg[g];
                   else if (!in_tile)
                     report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
                 }
               } else {
+                const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
                 // candidate mode: append the scores at or above the row's
                 // threshold, one atomic per warp and query (the warp's 32
                 // lanes hold 32 consecutive keys of the same query)
@@ -501,7 +516,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
                     if (ri >= 0 && ri < (long long)p.B * p.q_count) {
                       if (o < (unsigned int)p.cand_cap) {
                         p.cand_key[ri * p.cand_cap + o] = key;
-                        p.cand_idx[ri * p.cand_cap + o] = s * p.kstride;
+                        p.cand_idx[ri * p.cand_cap + o] = sp;
                       }
                     } else {
                       report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (3u << 8));
@@ -549,7 +564,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_I, (uint64_t)a.B * a.T * HI, DI, DI, kNSub, DI, sw))
     return cudaErrorInvalidValue;
-  IdxParams p;
+  IdxParams p = {};
   p.kv = a.kv;
   p.pool_rows = pool_rows;
   p.box_rows = box_rows;
@@ -596,10 +611,11 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   }
   const int grid = (int)(items < c.num_sms ? items : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<DI, HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       L::kAlloc);
+  const bool plain = ks == 1 && p.thr == nullptr && p.row_slot == nullptr;
+  auto kern = plain ? indexer_tc_kernel<DI, HI, true> : indexer_tc_kernel<DI, HI, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  indexer_tc_kernel<DI, HI><<<grid, EpiCfg<HI>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
+  kern<<<grid, EpiCfg<HI>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
   note_launches(1);
   return cudaGetLastError();
 }

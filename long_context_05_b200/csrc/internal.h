@@ -170,6 +170,8 @@ cudaError_t launch_wait_timeout_probe(const LaunchCtx& c);
 // shape validation and launch context of the public entry points (dsa_api.cu)
 dsa_status api_check_shape(const dsa_shape* s);
 dsa_status api_make_ctx(void* stream, LaunchCtx* c);
+// the key map (lengths, paged or contiguous caches) a shape describes
+KvMap api_kv_map(const dsa_shape* s);
 
 // split-k partial buffer size (floats) for a decode attention launch
 size_t attn_partial_floats(int rows, int H, int d_v, int nsplit);

@@ -36,8 +36,9 @@
 // TMEM accumulator is rescaled once (each softmax warp its half of the value
 // columns), after the previous P V has landed.
 //
-// Warp roles (480 threads): warp 0 owns TMEM and issues the MMAs (whichever
-// is ready: Q K^T of the next chunk or P V of the oldest), warps 1-3 and
+// Warp roles (512 threads): warp 0 owns TMEM and issues Q K^T of the even
+// chunks, warp 15 Q K^T of the odd chunks and every P V (one thread issuing
+// N = 64 MMAs back to back cannot keep the tensor pipe busy), warps 1-3 and
 // 12-14 gather, warps 4-11 run the softmax (thread = head row) and write the
 // output.  Decode splits the selected keys of each query over several CTAs
 // and merges the partial results with a combine kernel.  Every barrier that
@@ -64,7 +65,12 @@ constexpr int kSBuf = 2;        // S/P buffers in TMEM
 constexpr int kMmaWarp = 0, kFirstSoftmaxWarp = 4, kSoftmaxWarps = 8;
 constexpr int kGatherPerSlot = 3;
 constexpr int kFirstGatherB = kFirstSoftmaxWarp + kSoftmaxWarps;
-constexpr int kThreads = 32 * (kFirstGatherB + kGatherPerSlot);
+// A second MMA-issuing warp: one thread issuing back-to-back N = 64 MMAs
+// cannot keep the tensor pipe busy, so warp 0 issues Q K^T of the even
+// chunks and this warp Q K^T of the odd chunks and every P V (P V stays with
+// one thread: its accumulation into O must keep chunk order).
+constexpr int kMmaWarp2 = kFirstGatherB + kGatherPerSlot;
+constexpr int kThreads = 32 * (kMmaWarp2 + 1);
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -195,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], kSoftmaxWarps);
       mbar_init(&pv_done[i], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);   // one commit from each MMA-issuing warp
     for (int i = 0; i < kSBuf * 4 + 4; ++i) mbar_init(&mx_bar[i], 2);
     *abort_flag = 0;
     fence_mbar_init();
@@ -221,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return __all_sync(0xffffffffu, r);
   };
 
-  if (warp != kMmaWarp && (warp < kFirstSoftmaxWarp || warp >= kFirstGatherB)) {
+  if (warp != kMmaWarp && warp != kMmaWarp2 && (warp < kFirstSoftmaxWarp || warp >= kFirstGatherB)) {
     // ------------------------------------------------------------ gather
     // slot half h of every chunk; warp g of the half copies atoms g, g+3, g+6
     const int h = warp < kFirstSoftmaxWarp ? 0 : 1;
@@ -271,23 +277,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lanes 0, 8, 16, 24 hold rows 4m .. 4m+3
         const uint32_t bal = __ballot_sync(0xffffffffu, valid);
         mask |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u)) << (4 * m);
-        // an empty or invalid slot is zero-filled, so that no stale or
-        // non-finite shared memory meets its zero probability in P V
-        const uint16_t* src = p.kv + (size_t)(valid ? cr : 0) * DK;
+        // an empty or invalid slot is zero-filled (a copy that reads 0
+        // bytes), so that no stale or non-finite shared memory meets its zero
+        // probability in P V
+        const size_t crow = (size_t)(valid ? cr : 0);
+        const uint32_t nbytes = valid ? 16u : 0u;
+        const uint16_t* src = p.kv + crow * DK;
 #pragma unroll
         for (int a0 = 0; a0 < C::ATOMS; a0 += kGatherPerSlot) {
           const int a = a0 + g;
           uint8_t* dst = slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4);
           if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2) {
-            if (valid) cp_async16(dst, src + a * 64 + c16 * 8);
-            else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            cp_async16_zfill(dst, src + a * 64 + c16 * 8, nbytes);
           } else if (SEPV && a >= C::NATOM && a < C::ATOMS) {
             // value atom: columns half * DVH + (a - NATOM) * 64 .. of the value row
             const int vc = (a - C::NATOM) * 64 + c16 * 8;
-            if (vc < C::DVH) {
-              if (valid) cp_async16(dst, p.v + (size_t)cr * DV + half * C::DVH + vc);
-              else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-            }
+            if (vc < C::DVH) cp_async16_zfill(dst, p.v + crow * DV + half * C::DVH + vc, nbytes);
           }
         }
       }
@@ -301,9 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait<0>();
     // drain: the Q load must have landed before this CTA's memory is reused
     if (q_issued) mbar_wait(q_full, 0, p.wait_ns, no_abort);
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
     // ------------------------------------------------------------ MMA issue
+    // warp 0: Q K^T of even chunks; warp kMmaWarp2: Q K^T of odd chunks and
+    // all P V.  Chunk j uses S buffer j % 2 and ring slots 2 (j % NCH), +1.
     if (lane == 0) {
+      const int qk_par = warp == kMmaWarp ? 0 : 1;
+      const bool does_pv = warp == kMmaWarp2;
       constexpr uint32_t idesc_qk = make_idesc(kFmtBF16, kFmtBF16, 0, 0, 128, kN);
       constexpr uint32_t idesc_pv = make_idesc(kFmtBF16, kFmtBF16, 0, 1, 128, C::DVH);
       // descriptors are built once; a step only adds its byte offset >> 4 to
@@ -316,10 +325,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = nchunks == 0 || ((C::QS_ATOMS == 0 || mbar_wait(q_full, 0, p.wait_ns, ab)) &&
                                  mbar_wait(q_ready, 0, p.wait_ns, ab));
       if (!ok) fail(3);
-      // Issue whichever MMA is ready: Q K^T of chunk qk once its rows have
-      // landed and P V of chunk qk - kSBuf has freed its S buffer; P V of
-      // chunk pv once its probabilities are written.
-      int qk = 0, pv = 0;
+      // Issue whichever MMA of this thread is ready: Q K^T of chunk qk once
+      // its rows have landed and P V of chunk qk - kSBuf has freed its S
+      // buffer; P V of chunk pv once its probabilities are written (which
+      // implies Q K^T of pv has completed, whichever thread issued it).
+      int qk = qk_par, pv = 0;
+      int last_qk = -1;
       // P V of chunk pv: 4 K steps of 16 keys, A = P (TMEM), B = V (MN-major);
       // its commits free the chunk's S buffer and both ring slots
       auto issue_pv = [&]() {
@@ -339,9 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       uint64_t t_idle = 0;
       uint32_t spins = 0;
-      while (ok && pv < nchunks) {
+      while (ok && (qk < nchunks || (does_pv && pv < nchunks))) {
         bool progressed = false;
-        if (qk < nchunks && qk < pv + kSBuf) {
+        if (qk < nchunks) {
           const int s0 = (2 * qk) % kSlots, sb = qk % kSBuf;
           const uint32_t par = (uint32_t)((2 * qk) / kSlots) & 1;
           if (mbar_test_wait(&kv_full[s0], par) && mbar_test_wait(&kv_full[s0 + 1], par) &&
@@ -363,11 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             mma_commit(&s_full[sb]);
-            ++qk;
+            last_qk = qk;
+            qk += 2;
             progressed = true;
           }
         }
-        if (pv < qk && mbar_test_wait(&p_full[pv % kSBuf], (pv / kSBuf) & 1)) {
+        if (does_pv && pv < nchunks && mbar_test_wait(&p_full[pv % kSBuf], (pv / kSBuf) & 1)) {
           issue_pv();
           progressed = true;
         }
@@ -377,9 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // nothing ready: doze briefly on the event most likely next, with
         // bounded idle time, and abort when another role failed
-        if (pv < qk)
+        if (does_pv && pv < nchunks && (qk >= nchunks || pv < qk))
           mbar_try_wait_hint(&p_full[pv % kSBuf], (pv / kSBuf) & 1, 200);
-        else
+        else if (qk < nchunks)
           mbar_try_wait_hint(&kv_full[(2 * qk) % kSlots], (uint32_t)((2 * qk) / kSlots) & 1, 200);
         if (++spins == 1) t_idle = global_ns();
         if ((spins & 1023u) == 0u) {
@@ -391,16 +403,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // both issuers commit once: the phase completes when every MMA of
+      // both has finished
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
       // drain: the last arrivals of each commit barrier are not always waited
       // by their consumers; make sure they have landed before the CTA exits
-      for (int c = max(0, 2 * pv - kSlots); c < 2 * pv; ++c)
-        mbar_wait(&kv_empty[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
-      for (int i = max(0, pv - kSBuf); i < pv; ++i)
-        mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
-      for (int i = max(0, qk - kSBuf); i < qk; ++i)
-        mbar_wait(&s_full[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
+      if (does_pv) {
+        for (int c = max(0, 2 * pv - kSlots); c < 2 * pv; ++c)
+          mbar_wait(&kv_empty[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
+        for (int i = max(0, pv - kSBuf); i < pv; ++i)
+          mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
+      }
+      if (last_qk >= 0) mbar_wait(&s_full[last_qk % kSBuf], (last_qk / kSBuf) & 1, p.wait_ns, no_abort);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
@@ -634,7 +649,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, 
 template <int DK, int DV, bool SEPV>
 cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   using Cf = Cfg<DK, DV, SEPV>;
-  AttnParams p;
+  AttnParams p = {};
   p.map = a.map;
   p.q = a.q;
   p.kv = a.kv;

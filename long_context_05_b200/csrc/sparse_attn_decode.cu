@@ -217,8 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = sKV + a * kAtomBytes + kr * 128 + ((c16 ^ (kr & 7)) << 4);
         // an empty or invalid slot is zero-filled: no stale shared memory
         // meets its zero probability in P V
-        if (valid) cp_async16(dst, src + a * 64);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        cp_async16_zfill(dst, src + a * 64, valid ? 16u : 0u);
       }
     }
     if (sub == 0 && lane == 0) sMask[half] = mask;
@@ -507,7 +506,7 @@ bool attn_decode_supported(const AttnArgs& a) {
 cudaError_t launch_sparse_attn_decode(const LaunchCtx& c, const AttnArgs& a, void* part) {
   const long long rows = (long long)a.B * a.T;
   if (rows <= 0) return cudaSuccess;
-  DecParams p;
+  DecParams p = {};
   p.map = a.map;
   p.q = a.q;
   p.kv = a.kv;

@@ -76,7 +76,8 @@ extern "C" dsa_status dsa_topk_static(const dsa_shape* s, const float* scores, i
   if ((st = api_make_ctx(stream, &c)) != DSA_OK) return st;
   unsigned int* hist = nullptr;
   if ((st = static_hist(c.device, &hist)) != DSA_OK) return st;
-  TopkArgs a;
+  TopkArgs a = {};
+  a.kv = api_kv_map(s);
   a.scores = scores; a.ld = ld_scores; a.idx = idx;
   a.B = s->B; a.T = s->T; a.S = s->S; a.k = s->k;
   a.q_begin = q_begin; a.q_count = q_count;

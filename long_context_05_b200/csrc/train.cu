@@ -173,8 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 3; ++i) {
           const int a = sub + 3 * i;
           uint8_t* dst = sKV + a * kAtomBytes + kr * 128 + ((c16 ^ (kr & 7)) << 4);
-          if (valid) cp_async16(dst, src + a * 64);
-          else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          cp_async16_zfill(dst, src + a * 64, valid ? 16u : 0u);
         }
       }
     if (sub == 0 && lane == 0) sMask[half] = mask;
@@ -527,14 +526,8 @@ extern "C" dsa_status dsa_kl_target(const dsa_shape* s, const uint16_t* q, const
   LaunchCtx c;
   if ((st = api_make_ctx(stream, &c)) != DSA_OK) return st;
   if (q_count == 0) return DSA_OK;
-  TargetParams p;
-  p.map.seqlens = s->seqlens;
-  p.map.block_table = s->page_size > 0 ? s->block_table : nullptr;
-  p.map.S = s->S;
-  p.map.T = s->T;
-  p.map.page_size = s->page_size > 0 ? s->page_size : 0;
-  p.map.pages_per_seq = s->page_size > 0 ? s->pages_per_seq : 0;
-  p.map.num_pages = s->page_size > 0 ? s->num_pages : 0;
+  TargetParams p = {};
+  p.map = api_kv_map(s);
   p.q = q; p.kv = kv; p.lse = lse; p.idx = idx; p.target = target; p.ld = ld;
   p.T = s->T; p.H = s->H; p.k = s->k; p.q_begin = q_begin; p.q_count = q_count; p.B = s->B;
   const int slots = idx ? s->k : s->S;
@@ -564,9 +557,7 @@ extern "C" dsa_status dsa_indexer_kl(const dsa_shape* s, const float* scores, co
   LaunchCtx c;
   if ((st = api_make_ctx(stream, &c)) != DSA_OK) return st;
   if (q_count == 0) return DSA_OK;
-  KvMap map;
-  map.seqlens = s->seqlens; map.block_table = nullptr; map.S = s->S; map.T = s->T;
-  map.page_size = 0; map.pages_per_seq = 0; map.num_pages = 0;
+  const KvMap map = api_kv_map(s);
   indexer_kl_kernel<<<s->B * q_count, 256, 0, c.stream>>>(map, scores, target, ld, idx, s->T, s->k, q_begin, q_count,
                                                           grad, loss, c.err);
   note_launches(1);
@@ -584,13 +575,7 @@ extern "C" dsa_status dsa_indexer_backward(const dsa_shape* s, const uint8_t* q_
   LaunchCtx c;
   if ((st = api_make_ctx(stream, &c)) != DSA_OK) return st;
   if (q_count == 0) return DSA_OK;
-  KvMap map;
-  map.seqlens = s->seqlens;
-  map.block_table = s->page_size > 0 ? s->block_table : nullptr;
-  map.S = s->S; map.T = s->T;
-  map.page_size = s->page_size > 0 ? s->page_size : 0;
-  map.pages_per_seq = s->page_size > 0 ? s->pages_per_seq : 0;
-  map.num_pages = s->page_size > 0 ? s->num_pages : 0;
+  const KvMap map = api_kv_map(s);
   cudaError_t e = cudaErrorInvalidValue;
 #define DSA_BWD(HI_, DI_)                                                                                          \
   if (s->H_I == HI_ && s->D_I == DI_)                                                                              \

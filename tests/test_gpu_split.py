@@ -67,9 +67,10 @@ def test_key_split_decode(parts):
     out, lse = computes[0].combine(o_all, l_all)
     st, det = dsa.device_error()
     assert st == 0, (st, hex(det))
+    # every part merges to the same selection (as sets: slot order is free)
     gidx = merged[0][0].cpu().numpy()
     for m in merged[1:]:
-        assert torch.equal(m[0], merged[0][0])
+        assert torch.equal(torch.sort(m[0], dim=-1).values, torch.sort(merged[0][0], dim=-1).values)
     ref_idx = ref.idx.cpu().numpy()[:, 0]
     og, lg = out.float().cpu().numpy()[:, 0], lse.cpu().numpy()[:, 0]
     stats = P.ErrStats()
