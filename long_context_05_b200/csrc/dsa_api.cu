@@ -129,6 +129,9 @@ float tau_of(const dsa_shape* s) {
 // contiguous key cache (the sample reads every kSampleStride-th cache row).
 constexpr int kSampleStride = 16;
 constexpr int kRepairRows = 64;   // rows of one block that can fall back to a materialised score row
+constexpr int kTargetNum = 3, kTargetDen = 2;   // about 1.5 k candidates expected per row
+constexpr int kRowCap = 6144;     // candidates a row's list holds (<= the top-k's shared capacity)
+constexpr int kWarpSlack = 2;     // warp lists hold twice the expected candidates
 
 bool fused_select(const dsa_shape* s) {
   return s->mode == DSA_PREFILL && s->page_size == 0 && s->S % kSampleStride == 0 &&
@@ -139,14 +142,18 @@ bool fused_select(const dsa_shape* s) {
 //   [score tile, or the fused selection's regions][attention split partials]
 //   [top-k histograms]
 // The fused selection's regions, for R = B * q_rows rows: the key-sample
-// tile [R, ld_s] FP32, thresholds, candidate counts and repair slots [R],
-// candidate keys and indices [R, cap], the repair list and its count, and
-// the repair tile [kRepairRows, ld] FP32.
+// tile [R, ld_s] FP32; thresholds, candidate counts, repair slots and
+// overflow flags [R]; the indexer warps' candidate lists (row, index, key)
+// [nwl, wl_cap] and their counts [nwl]; the per-row candidate keys and
+// indices [R, cap]; the repair list and its count; the repair tile
+// [kRepairRows, ld] FP32.
 struct WsLayout {
   bool fused;
-  size_t sample_off, thr_off, cnt_off, slot_off, ckey_off, cidx_off, fail_off, nfail_off, repair_off;
+  size_t sample_off, thr_off, cnt_off, slot_off, rfail_off, wrow_off, widx_off, wkey_off, wcnt_off, ckey_off,
+      cidx_off, fail_off, nfail_off, repair_off;
   int64_t ld_s;
-  int cap;
+  int cap, nwl;
+  long long wl_cap;
   size_t scores_off, scores_bytes;
   size_t part_off, part_bytes;
   size_t topk_off, topk_bytes;
@@ -160,15 +167,26 @@ WsLayout ws_layout(const dsa_shape* s, int num_sms) {
   L.q_rows = s->mode == DSA_DECODE ? s->T : q_block_of(s);
   L.scores_off = 0;
   L.fused = fused_select(s);
-  L.cap = topk_cand_cap();
+  L.cap = kRowCap < topk_cand_cap() ? kRowCap : topk_cand_cap();
   L.ld_s = (int64_t)round_up((size_t)(s->S / kSampleStride), 64);
   if (L.fused) {
     const size_t R = (size_t)s->B * L.q_rows;
+    // one list per indexer epilogue warp (a persistent grid of at most one
+    // CTA per SM), together kWarpSlack times the expected candidates
+    L.nwl = num_sms * indexer_epilogue_warps(s->H_I);
+    const long long expect = (long long)R * s->k * kTargetNum / kTargetDen;
+    L.wl_cap = (expect * kWarpSlack + L.nwl - 1) / L.nwl;
+    const size_t W = (size_t)L.nwl * L.wl_cap;
     size_t o = 0;
     L.sample_off = o; o += round_up(R * L.ld_s * sizeof(float), 256);
     L.thr_off = o; o += round_up(R * 4, 256);
     L.cnt_off = o; o += round_up(R * 4, 256);
     L.slot_off = o; o += round_up(R * 4, 256);
+    L.rfail_off = o; o += round_up(R * 4, 256);
+    L.wrow_off = o; o += round_up(W * 4, 256);
+    L.widx_off = o; o += round_up(W * 4, 256);
+    L.wkey_off = o; o += round_up(W * 4, 256);
+    L.wcnt_off = o; o += round_up((size_t)L.nwl * 4, 256);
     L.ckey_off = o; o += round_up(R * L.cap * 4, 256);
     L.cidx_off = o; o += round_up(R * L.cap * 4, 256);
     L.fail_off = o; o += round_up(kRepairRows * 4, 256);
@@ -233,6 +251,11 @@ dsa_status run_select_fused(const LaunchCtx& c, const dsa_shape* s, const WsLayo
   unsigned int* thr = reinterpret_cast<unsigned int*>(ws + L.thr_off);
   unsigned int* ccnt = reinterpret_cast<unsigned int*>(ws + L.cnt_off);
   int* slot = reinterpret_cast<int*>(ws + L.slot_off);
+  int* rfail = reinterpret_cast<int*>(ws + L.rfail_off);
+  int32_t* wrow = reinterpret_cast<int32_t*>(ws + L.wrow_off);
+  int32_t* widx = reinterpret_cast<int32_t*>(ws + L.widx_off);
+  unsigned int* wkey = reinterpret_cast<unsigned int*>(ws + L.wkey_off);
+  unsigned int* wcnt = reinterpret_cast<unsigned int*>(ws + L.wcnt_off);
   unsigned int* ckey = reinterpret_cast<unsigned int*>(ws + L.ckey_off);
   int32_t* cidx = reinterpret_cast<int32_t*>(ws + L.cidx_off);
   int* fail = reinterpret_cast<int*>(ws + L.fail_off);
@@ -260,22 +283,29 @@ dsa_status run_select_fused(const LaunchCtx& c, const dsa_shape* s, const WsLayo
     sa.ld = L.ld_s;
     if ((e = launch_indexer(c, sa)) != cudaSuccess) return DSA_ERR_CUDA;
   }
-  // 2. per-row thresholds (about 2k expected candidates), counts cleared
-  if ((e = launch_topk_threshold(c, ta, sample, L.ld_s, kSampleStride, 2 * s->k, thr, ccnt, slot, nfail)) !=
-      cudaSuccess)
+  // 2. per-row thresholds (about 1.5 k expected candidates); counts,
+  //    flags and the warp lists' lengths cleared
+  if ((e = launch_topk_threshold(c, ta, sample, L.ld_s, kSampleStride, s->k * kTargetNum / kTargetDen, L.cap, thr, ccnt,
+                                 slot, rfail, nfail, wcnt, L.nwl)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  // 3. every key scored, candidates appended
+  // 3. every key scored; each epilogue warp appends its candidates to its own list
   IndexerArgs ca = ia;
   ca.thr = thr;
-  ca.cand_key = ckey;
-  ca.cand_idx = cidx;
-  ca.cand_cnt = ccnt;
-  ca.cand_cap = L.cap;
+  ca.wl_row = wrow;
+  ca.wl_idx = widx;
+  ca.wl_key = wkey;
+  ca.wl_cnt = wcnt;
+  ca.wl_cap = L.wl_cap;
+  ca.row_fail = rfail;
   if ((e = launch_indexer(c, ca)) != cudaSuccess) return DSA_ERR_CUDA;
-  // 4. exact selection among the candidates
-  if ((e = launch_topk_cand_select(c, ta, ckey, cidx, ccnt, L.cap, slot, fail, nfail, kRepairRows)) != cudaSuccess)
+  // 4. the warp lists into per-row lists
+  if ((e = launch_topk_scatter(c, wrow, widx, wkey, wcnt, L.wl_cap, L.nwl, ccnt, ckey, cidx, L.cap)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  // 5. repair (both launches return at once when no row was listed)
+  // 5. exact selection among each row's candidates
+  if ((e = launch_topk_cand_select(c, ta, ckey, cidx, ccnt, L.cap, rfail, slot, fail, nfail, kRepairRows)) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  // 6. repair (both launches return at once when no row was listed)
   IndexerArgs ra = ia;
   ra.row_slot = slot;
   ra.scores = repair;

@@ -64,10 +64,12 @@ struct IdxParams {
   int box_rows;        // key rows per TMA load (a key tile takes kBM / box_rows)
   int kstride;         // column s of a score row is key s * kstride (1: every key)
   const unsigned int* thr;   // candidate mode: per launch row, the smallest order key kept
-  unsigned int* cand_key;
-  int32_t* cand_idx;
-  unsigned int* cand_cnt;
-  int cand_cap;
+  int32_t* wl_row;           // candidate lists, one per epilogue warp of the launch
+  int32_t* wl_idx;
+  unsigned int* wl_key;
+  unsigned int* wl_cnt;
+  long long wl_cap;
+  int* row_fail;
   const int* row_slot;       // repair mode: score row of each launch row (-1: skip)
   const float* w;
   const float* q_scale;
@@ -165,9 +167,10 @@ __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, 
   return j < 0 ? 0 : (j < nsub - 1 ? j : nsub - 1);
 }
 
-// PLAIN: every key scored into score rows (stride 1, no thresholds, no repair
-// list); the general form adds the key sample, the candidate and the repair
-// modes, whose per-element checks the plain form must not pay.
+// PLAIN: every key of a contiguous cache scored into score rows (stride 1,
+// no thresholds, no repair list); the general form adds paged caches, the key
+// sample, the candidate and the repair modes, whose checks the plain form
+// must not pay.
 template <int DI, int HI, bool PLAIN>
 __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
             // a key sample is a contiguous cache read every kstride-th row:
             // row b * (S / kstride) + sample index of the strided map
             long long y = s >= it.L ? -1
-                          : KS == 1 ? p.kv.row(it.b, s)
+                          : KS == 1 ? p.kv.row<!PLAIN>(it.b, s)
                                            : (long long)it.b * (p.S / KS) + kt * kBM + r0;
             if (y < 0) {
               if (s < it.L) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (2u << 8));
@@ -371,6 +374,9 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     const int r = quarter * 32 + lane;   // key row within a tile
     const int etid = threadIdx.x - 64;
     uint32_t u = 0, items = 0;
+    // candidate mode: this warp's list and its length (warp-uniform)
+    const long long wl0 = ((long long)blockIdx.x * (E::EPI_THREADS / 32) + ew) * p.wl_cap;
+    long long wpos = 0;
     for_each_item<HI, PLAIN>(p, [&](const Item& it) {
       // per-item head weights  wM[(query, head)] = w * q_scale  (0 past the end)
       float* wbuf = sW + (items & 1) * L::kWFloats;
@@ -405,7 +411,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           sg[g] = (kt + g) * kBM + r;
           // 1/2: the head sum below accumulates 2 ReLU(x)
           spos[g] = sg[g] * KS;   // key position of column sg[g]
-          const long long kr = (g < ng && spos[g] < it.L) ? p.kv.row(it.b, spos[g]) : -1;
+          const long long kr = (g < ng && spos[g] < it.L) ? p.kv.row<!PLAIN>(it.b, spos[g]) : -1;
           ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
         }
         const int jlo = first_active<HI, PLAIN>(p, it, kt, nsub);
@@ -501,28 +507,27 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
               } else {
                 const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
                 // candidate mode: append the scores at or above the row's
-                // threshold, one atomic per warp and query (the warp's 32
-                // lanes hold 32 consecutive keys of the same query)
+                // threshold to this warp's own list (the 32 lanes hold 32
+                // consecutive keys of the same query: a ballot gives each
+                // taking lane its slot, with no atomic)
                 const unsigned int key = order_key(a * ksg[g]);
                 const bool take = vis && key >= tq[j * QPS + q];
                 const unsigned int m = __ballot_sync(0xffffffffu, take);
-                if (m != 0u) {
-                  const int leader = __ffs(m) - 1;
-                  unsigned int base = 0;
-                  if (lane == leader) base = atomicAdd(&p.cand_cnt[ri], (unsigned int)__popc(m));
-                  base = __shfl_sync(0xffffffffu, base, leader);
-                  if (take) {
-                    const unsigned int o = base + (unsigned int)__popc(m & ((1u << lane) - 1u));
-                    if (ri >= 0 && ri < (long long)p.B * p.q_count) {
-                      if (o < (unsigned int)p.cand_cap) {
-                        p.cand_key[ri * p.cand_cap + o] = key;
-                        p.cand_idx[ri * p.cand_cap + o] = sp;
-                      }
+                if (take) {
+                  const long long o = wpos + __popc(m & ((1u << lane) - 1u));
+                  if (ri >= 0 && ri < (long long)p.B * p.q_count) {
+                    if (o < p.wl_cap) {
+                      p.wl_row[wl0 + o] = (int32_t)ri;
+                      p.wl_idx[wl0 + o] = sp;
+                      p.wl_key[wl0 + o] = key;
                     } else {
-                      report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (3u << 8));
+                      p.row_fail[ri] = 1;   // dropped: the row is repaired later
                     }
+                  } else {
+                    report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (3u << 8));
                   }
                 }
+                wpos += __popc(m);
               }
             }
           }
@@ -530,6 +535,8 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       }
       return true;
     });
+    if (THR != nullptr && lane == 0)
+      p.wl_cnt[blockIdx.x * (E::EPI_THREADS / 32) + ew] = (unsigned int)(wpos < p.wl_cap ? wpos : p.wl_cap);
   }
 
   tc_fence_before();
@@ -570,10 +577,12 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   p.box_rows = box_rows;
   p.kstride = ks;
   p.thr = a.thr;
-  p.cand_key = a.cand_key;
-  p.cand_idx = a.cand_idx;
-  p.cand_cnt = a.cand_cnt;
-  p.cand_cap = a.cand_cap;
+  p.wl_row = a.wl_row;
+  p.wl_idx = a.wl_idx;
+  p.wl_key = a.wl_key;
+  p.wl_cnt = a.wl_cnt;
+  p.wl_cap = a.wl_cap;
+  p.row_fail = a.row_fail;
   p.row_slot = a.row_slot;
   p.w = a.w;
   p.q_scale = a.q_scale;
@@ -611,7 +620,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   }
   const int grid = (int)(items < c.num_sms ? items : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  const bool plain = ks == 1 && p.thr == nullptr && p.row_slot == nullptr;
+  const bool plain = ks == 1 && p.thr == nullptr && p.row_slot == nullptr && a.kv.page_size == 0;
   auto kern = plain ? indexer_tc_kernel<DI, HI, true> : indexer_tc_kernel<DI, HI, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
@@ -633,6 +642,8 @@ cudaError_t launch_di(const LaunchCtx& c, const IndexerArgs& a) {
 }
 
 }  // namespace
+
+int indexer_epilogue_warps(int H_I) { return (H_I >= 32 ? EpiCfg<64>::EPI_THREADS : EpiCfg<4>::EPI_THREADS) / 32; }
 
 cudaError_t launch_indexer(const LaunchCtx& c, const IndexerArgs& a) {
   if (a.q_count <= 0 || a.B <= 0) return cudaSuccess;

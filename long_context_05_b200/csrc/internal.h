@@ -60,9 +60,14 @@ struct KvMap {
     }
     return L;
   }
+  // Cache row of token s of sequence b in a contiguous [B, S, ...] cache.
+  __device__ __forceinline__ long long row_contig(int b, int s) const { return (long long)b * S + s; }
   // Cache row of token s of sequence b, or -1 when its page is not mapped.
+  // Kernels instantiate a contiguous form that calls row_contig instead, so
+  // that the page lookup stays out of their hot loops.
+  template <bool PAGED = true>
   __device__ __forceinline__ long long row(int b, int s) const {
-    if (page_size == 0) return (long long)b * S + s;
+    if (!PAGED || page_size == 0) return (long long)b * S + s;
     const int pg = s / page_size;
     if (pg < 0 || pg >= pages_per_seq) return -1;
     const int e = block_table[(size_t)b * pages_per_seq + pg];
@@ -88,14 +93,18 @@ struct LaunchCtx {
 struct IndexerArgs {
   KvMap kv;
   int kstride;              // score every kstride-th key only (a sample; contiguous caches, S % kstride == 0)
-  // candidate mode (thr set): instead of writing score rows, append the
-  // (order key, key index) of every visible score whose key is >= thr[row]
-  // to row's list of cand_cap slots, counting in cand_cnt[row]
+  // candidate mode (thr set): instead of writing score rows, every epilogue
+  // warp appends (launch row, key index, order key) of each visible score
+  // whose key is >= thr[row] to its own list of wl_cap entries (warp w of the
+  // launch at w * wl_cap; no atomics), and writes its count to wl_cnt[w];
+  // entries past wl_cap are dropped and their rows flagged in row_fail
   const unsigned int* thr;
-  unsigned int* cand_key;
-  int32_t* cand_idx;
-  unsigned int* cand_cnt;
-  int cand_cap;
+  int32_t* wl_row;
+  int32_t* wl_idx;
+  unsigned int* wl_key;
+  unsigned int* wl_cnt;
+  long long wl_cap;
+  int* row_fail;
   // repair mode (row_slot set): score only the rows with row_slot[row] >= 0,
   // into score row row_slot[row]; work items without such a row are skipped
   const int* row_slot;
@@ -157,11 +166,18 @@ int topk_merge_max_candidates();
 // candidate modes feed it)
 int topk_cand_cap();
 cudaError_t launch_topk_threshold(const LaunchCtx& c, const TopkArgs& a, const float* sample, long long ld_s,
-                                  int kstride, int target, unsigned int* thr, unsigned int* cnt, int* row_slot,
-                                  unsigned int* nfail);
+                                  int kstride, int target, int cap, unsigned int* thr, unsigned int* cnt, int* row_slot,
+                                  int* row_fail, unsigned int* nfail, unsigned int* wl_cnt, int nwl);
 cudaError_t launch_topk_cand_select(const LaunchCtx& c, const TopkArgs& a, const unsigned int* cand_key,
-                                    const int32_t* cand_idx, const unsigned int* cnt, int cap, int* row_slot,
-                                    int* fail_rows, unsigned int* nfail, int max_fail);
+                                    const int32_t* cand_idx, const unsigned int* cnt, int cap, const int* row_fail,
+                                    int* row_slot, int* fail_rows, unsigned int* nfail, int max_fail);
+// the warps' candidate lists into per-row lists [rows, cap] (counts in cnt)
+cudaError_t launch_topk_scatter(const LaunchCtx& c, const int32_t* wl_row, const int32_t* wl_idx,
+                                const unsigned int* wl_key, const unsigned int* wl_cnt, long long wl_cap, int nwarps,
+                                unsigned int* cnt, unsigned int* cand_key, int32_t* cand_idx, int cap);
+// epilogue warps of one indexer CTA, and the indexer's grid, for sizing its
+// candidate lists
+int indexer_epilogue_warps(int H_I);
 cudaError_t launch_topk_repair(const LaunchCtx& c, const TopkArgs& a, const float* tile, long long ld,
                                const int* fail_rows, const unsigned int* nfail, int max_fail);
 

@@ -142,7 +142,9 @@ struct AttnParams {
 
 
 
-template <int DK, int DV, bool SEPV>
+// PAGED: the caches are page pools (block table lookup per gathered key);
+// the contiguous form computes the row directly.
+template <int DK, int DV, bool SEPV, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, AttnParams p) {
   using C = Cfg<DK, DV, SEPV>;
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
           v = -1;
         }
-        long long cr = v >= 0 ? p.map.row(b, v) : -1;   // cache row of key v
+        long long cr = v >= 0 ? p.map.row<PAGED>(b, v) : -1;   // cache row of key v
         if (v >= 0 && cr < 0) {
           if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
           v = -1;
@@ -337,11 +339,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int s0 = (2 * pv) % kSlots, sb = pv % kSBuf;
         const uint64_t vst = vdesc0 + (uint64_t)((s0 * C::SLOT_ATOM) >> 4);
+        if (!SEPV) {
 #pragma unroll
-        for (int ks = 0; ks < kN / 16; ++ks) {
-          const uint64_t vdesc = vst + (uint64_t)((ks * 16 * 128) >> 4);
-          mma_bf16_ts(tmem + C::OCOL, tmem + C::SCOL + sb * kN + ks * 8, vdesc, idesc_pv,
-                      (pv > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < kN / 16; ++ks) {
+            const uint64_t vdesc = vst + (uint64_t)((ks * 16 * 128) >> 4);
+            mma_bf16_ts(tmem + C::OCOL, tmem + C::SCOL + sb * kN + ks * 8, vdesc, idesc_pv,
+                        (pv > 0 || ks > 0) ? 1u : 0u);
+          }
+        } else {
+          // values in their own atoms: one N = 64 MMA per 64-column atom
+          constexpr uint32_t idesc_pv64 = make_idesc(kFmtBF16, kFmtBF16, 0, 1, 128, 64);
+#pragma unroll
+          for (int nb = 0; nb < C::NVATOM; ++nb)
+#pragma unroll
+            for (int ks = 0; ks < kN / 16; ++ks) {
+              const uint64_t vdesc = vst + (uint64_t)((nb * C::ATOM_STRIDE + ks * 16 * 128) >> 4);
+              mma_bf16_ts(tmem + C::OCOL + nb * 64, tmem + C::SCOL + sb * kN + ks * 8, vdesc, idesc_pv64,
+                          (pv > 0 || ks > 0) ? 1u : 0u);
+            }
         }
         mma_commit(&pv_done[sb]);
         mma_commit(&kv_empty[s0]);
@@ -646,7 +661,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, 
     lse[(size_t)row * H + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int DK, int DV, bool SEPV>
+template <int DK, int DV, bool SEPV, bool PAGED>
 cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   using Cf = Cfg<DK, DV, SEPV>;
   AttnParams p = {};
@@ -678,11 +693,11 @@ cudaError_t launch_tc(const LaunchCtx& c, const AttnArgs& a) {
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, (uint64_t)rows * a.H, DK, (uint64_t)DK * 2, 128,
                     64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<DK, DV, SEPV>,
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<DK, DV, SEPV, PAGED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (e != cudaSuccess) return e;
   const long long ctas = rows * a.nsplit * Cf::NHALF;
-  sparse_attn_tc_kernel<DK, DV, SEPV><<<(unsigned)ctas, kThreads, Cf::ALLOC, c.stream>>>(tm_q, p);
+  sparse_attn_tc_kernel<DK, DV, SEPV, PAGED><<<(unsigned)ctas, kThreads, Cf::ALLOC, c.stream>>>(tm_q, p);
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.nsplit == 1) return e;
@@ -714,9 +729,15 @@ int attn_choose_nsplit(int rows, int H, int d_v, int k, int num_sms) {
 cudaError_t launch_sparse_attn(const LaunchCtx& c, const AttnArgs& a) {
   if ((long long)a.B * a.T <= 0) return cudaSuccess;
   if (a.nsplit > 1 && a.part == nullptr) return cudaErrorInvalidValue;
-  const bool sepv = a.v != nullptr;
-  if (a.d_k == 576 && a.d_v == 512) return sepv ? launch_tc<576, 512, true>(c, a) : launch_tc<576, 512, false>(c, a);
-  if (a.d_k == 80 && a.d_v == 64) return sepv ? launch_tc<80, 64, true>(c, a) : launch_tc<80, 64, false>(c, a);
+  const bool sepv = a.v != nullptr, paged = a.map.page_size != 0;
+  if (a.d_k == 576 && a.d_v == 512) {
+    if (paged) return sepv ? launch_tc<576, 512, true, true>(c, a) : launch_tc<576, 512, false, true>(c, a);
+    return sepv ? launch_tc<576, 512, true, false>(c, a) : launch_tc<576, 512, false, false>(c, a);
+  }
+  if (a.d_k == 80 && a.d_v == 64) {
+    if (paged) return sepv ? launch_tc<80, 64, true, true>(c, a) : launch_tc<80, 64, false, true>(c, a);
+    return sepv ? launch_tc<80, 64, true, false>(c, a) : launch_tc<80, 64, false, false>(c, a);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -93,6 +93,7 @@ struct DecParams {
   DevErr* err;
 };
 
+template <bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, DecParams p) {
   extern __shared__ uint8_t smem[];
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c16 == 0 && sub == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
         v = -1;
       }
-      const long long cr = v >= 0 ? p.map.row(b, v) : -1;
+      const long long cr = v >= 0 ? p.map.row<PAGED>(b, v) : -1;
       if (v >= 0 && cr < 0) {
         if (c16 == 0 && sub == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
         v = -1;
@@ -531,9 +532,10 @@ cudaError_t launch_sparse_attn_decode(const LaunchCtx& c, const AttnArgs& a, voi
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, (uint64_t)rows * a.H, DK, (uint64_t)DK * 2, 128,
                     64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  auto kern = a.map.page_size != 0 ? sparse_attn_decode_kernel<true> : sparse_attn_decode_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  sparse_attn_decode_kernel<<<(unsigned)(rows * p.nsplit), kThreads, kSmem, c.stream>>>(tm_q, p);
+  kern<<<(unsigned)(rows * p.nsplit), kThreads, kSmem, c.stream>>>(tm_q, p);
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.nsplit == 1) return e;

@@ -471,10 +471,12 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, DevEr
 // candidates fall short or overflow are listed for repair: the indexer scores
 // just those rows into a small tile and select_row finishes them.
 
-// Threshold per row, its candidate count cleared, its repair slot unset.
+// Threshold per row, its candidate count and overflow flag cleared, its
+// repair slot unset (block 0 also clears the repair count).
 __global__ void __launch_bounds__(kThreads, 2)
-    topk_threshold_kernel(TopkArgs a, const float* sample, long long ld_s, int kstride, int target,
-                          unsigned int* thr, unsigned int* cnt, int* row_slot, unsigned int* nfail, DevErr* err) {
+    topk_threshold_kernel(TopkArgs a, const float* sample, long long ld_s, int kstride, int target, int cap,
+                          unsigned int* thr, unsigned int* cnt, int* row_slot, int* row_fail, unsigned int* nfail,
+                          unsigned int* wl_cnt, int nwl, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int r = blockIdx.x;
@@ -485,9 +487,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     cnt[r] = 0u;
     row_slot[r] = -1;
+    row_fail[r] = 0;
     if (r == 0) *nfail = 0u;
   }
-  if (n <= kCap) {  // the candidate list holds every visible key
+  // warp lists the indexer's grid may leave unwritten read as empty
+  if (r == 0)
+    for (int i = threadIdx.x; i < nwl; i += kThreads) wl_cnt[i] = 0u;
+  if (n <= cap) {  // the candidate list holds every visible key
     if (threadIdx.x == 0) thr[r] = 0u;
     return;
   }
@@ -515,8 +521,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 // allow in the meantime).
 __global__ void __launch_bounds__(kThreads, 2)
     topk_cand_select_kernel(TopkArgs a, const unsigned int* cand_key, const int32_t* cand_idx,
-                            const unsigned int* cnt, int cap, int* row_slot, int* fail_rows, unsigned int* nfail,
-                            int max_fail, DevErr* err) {
+                            const unsigned int* cnt, int cap, const int* row_fail, int* row_slot, int* fail_rows,
+                            unsigned int* nfail, int max_fail, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int r = blockIdx.x;
@@ -530,7 +536,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   const unsigned int c = cnt[r];
-  const bool complete = c >= (unsigned int)k && c <= (unsigned int)cap && c <= (unsigned int)kCap;
+  const bool complete =
+      c >= (unsigned int)k && c <= (unsigned int)cap && c <= (unsigned int)kCap && row_fail[r] == 0;
   const int nc = (int)min(c, (unsigned int)min(cap, kCap));
   for (int i = threadIdx.x; i < nc; i += kThreads) {
     sm.ck[i] = cand_key[(size_t)r * cap + i];
@@ -549,6 +556,25 @@ __global__ void __launch_bounds__(kThreads, 2)
       row_slot[r] = (int)slot;
     } else {
       report_error(err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_TOPK | (0x40u << 8));
+    }
+  }
+}
+
+// The epilogue warps' candidate lists into per-row lists: one block per
+// warp list, one returning atomic per entry (latency hidden by the many
+// blocks in flight, away from the indexer's epilogue).
+__global__ void __launch_bounds__(256)
+    topk_scatter_kernel(const int32_t* wl_row, const int32_t* wl_idx, const unsigned int* wl_key,
+                        const unsigned int* wl_cnt, long long wl_cap, unsigned int* cnt, unsigned int* cand_key,
+                        int32_t* cand_idx, int cap) {
+  const long long base = (long long)blockIdx.x * wl_cap;
+  const long long n = min((long long)wl_cnt[blockIdx.x], wl_cap);
+  for (long long i = threadIdx.x; i < n; i += 256) {
+    const int r = wl_row[base + i];
+    const unsigned int pos = atomicAdd(&cnt[r], 1u);
+    if (pos < (unsigned int)cap) {
+      cand_key[(size_t)r * cap + pos] = wl_key[base + i];
+      cand_idx[(size_t)r * cap + pos] = wl_idx[base + i];
     }
   }
 }
@@ -877,29 +903,39 @@ int topk_merge_max_candidates() { return kCap; }
 int topk_cand_cap() { return kCap; }
 
 cudaError_t launch_topk_threshold(const LaunchCtx& c, const TopkArgs& a, const float* sample, long long ld_s,
-                                  int kstride, int target, unsigned int* thr, unsigned int* cnt, int* row_slot,
-                                  unsigned int* nfail) {
+                                  int kstride, int target, int cap, unsigned int* thr, unsigned int* cnt, int* row_slot,
+                                  int* row_fail, unsigned int* nfail, unsigned int* wl_cnt, int nwl) {
   const int rows = a.B * a.q_count;
   if (rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(topk_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_threshold_kernel<<<rows, kThreads, smem, c.stream>>>(a, sample, ld_s, kstride, target, thr, cnt, row_slot,
-                                                            nfail, c.err);
+  topk_threshold_kernel<<<rows, kThreads, smem, c.stream>>>(a, sample, ld_s, kstride, target, cap, thr, cnt, row_slot,
+                                                            row_fail, nfail, wl_cnt, nwl, c.err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_scatter(const LaunchCtx& c, const int32_t* wl_row, const int32_t* wl_idx,
+                                const unsigned int* wl_key, const unsigned int* wl_cnt, long long wl_cap, int nwarps,
+                                unsigned int* cnt, unsigned int* cand_key, int32_t* cand_idx, int cap) {
+  if (nwarps <= 0) return cudaSuccess;
+  topk_scatter_kernel<<<nwarps, 256, 0, c.stream>>>(wl_row, wl_idx, wl_key, wl_cnt, wl_cap, cnt, cand_key, cand_idx,
+                                                    cap);
   note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topk_cand_select(const LaunchCtx& c, const TopkArgs& a, const unsigned int* cand_key,
-                                    const int32_t* cand_idx, const unsigned int* cnt, int cap, int* row_slot,
-                                    int* fail_rows, unsigned int* nfail, int max_fail) {
+                                    const int32_t* cand_idx, const unsigned int* cnt, int cap, const int* row_fail,
+                                    int* row_slot, int* fail_rows, unsigned int* nfail, int max_fail) {
   const int rows = a.B * a.q_count;
   if (rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(topk_cand_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_cand_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, cand_key, cand_idx, cnt, cap, row_slot, fail_rows,
-                                                              nfail, max_fail, c.err);
+  topk_cand_select_kernel<<<rows, kThreads, smem, c.stream>>>(a, cand_key, cand_idx, cnt, cap, row_fail, row_slot,
+                                                              fail_rows, nfail, max_fail, c.err);
   note_launches(1);
   return cudaGetLastError();
 }
