@@ -125,7 +125,7 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
     const int g = gid - b * p.groups_per_seq;
     Item it;
     it.b = b;
-    it.L = p.kv.len(b, p.err, ERR_SITE_INDEXER);
+    it.L = PLAIN ? p.S : p.kv.len(b, p.err, ERR_SITE_INDEXER);
     it.off = it.L - p.T;
     it.t0 = p.q_begin + g * per_group;
     it.tend = min(it.t0 + per_group, q_end);
@@ -167,10 +167,10 @@ __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, 
   return j < 0 ? 0 : (j < nsub - 1 ? j : nsub - 1);
 }
 
-// PLAIN: every key of a contiguous cache scored into score rows (stride 1,
-// no thresholds, no repair list); the general form adds paged caches, the key
-// sample, the candidate and the repair modes, whose checks the plain form
-// must not pay.
+// PLAIN: every key of a contiguous cache of S keys per sequence scored into
+// score rows (no per-sequence lengths, stride 1, no thresholds, no repair
+// list); the general form adds lengths, paged caches, the key sample, the
+// candidate and the repair modes, whose checks the plain form must not pay.
 template <int DI, int HI, bool PLAIN>
 __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -272,6 +272,9 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           // the tile's keys in runs of box_rows cache rows (a whole tile when
           // the cache is contiguous); a run at or past L_b, or on an unmapped
           // page, reads the fill value from past the end of the pool
+          if constexpr (PLAIN) {
+            tma_load_2d(sA + st * L::kABytes, &tm_k, &a_full[st], 0, it.b * p.S + kt * kBM);
+          } else {
           for (int r0 = 0; r0 < kBM; r0 += p.box_rows) {
             const int s = (kt * kBM + r0) * KS;
             // a key sample is a contiguous cache read every kstride-th row:
@@ -284,6 +287,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
               y = p.pool_rows;
             }
             tma_load_2d(sA + st * L::kABytes + r0 * DI, &tm_k, &a_full[st], 0, (int)y);
+          }
           }
           issued[st] = true;
           last_phase[st] = (a_cnt / kStages) & 1;
@@ -411,8 +415,12 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           sg[g] = (kt + g) * kBM + r;
           // 1/2: the head sum below accumulates 2 ReLU(x)
           spos[g] = sg[g] * KS;   // key position of column sg[g]
-          const long long kr = (g < ng && spos[g] < it.L) ? p.kv.row<!PLAIN>(it.b, spos[g]) : -1;
-          ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
+          if constexpr (PLAIN) {
+            ksg[g] = (g < ng && sg[g] < p.S) ? 0.5f * p.k_scale[(size_t)it.b * p.S + sg[g]] : 0.f;
+          } else {
+            const long long kr = (g < ng && spos[g] < it.L) ? p.kv.row<true>(it.b, spos[g]) : -1;
+            ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
+          }
         }
         const int jlo = first_active<HI, PLAIN>(p, it, kt, nsub);
         const uint32_t u0 = u;
@@ -493,7 +501,16 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
               for (int i = 0; i < NP; ++i) a += part[g][q][i].x + part[g][q][i].y;
               const int t = it.t0 + j * QPS + q;
               const bool vis = t < it.tend && sp <= it.off + t;
-              if (THR == nullptr) {
+              if constexpr (PLAIN) {
+                if (vis) {
+                  // self-check: the score slot lies inside this launch's tile
+                  const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
+                  if (ri >= 0 && ri < (long long)p.B * p.q_count && s >= 0 && s < p.ld)
+                    p.scores[ri * p.ld + s] = a * ksg[g];
+                  else
+                    report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
+                }
+              } else if (THR == nullptr) {
                 if (vis) {
                   // self-check: the score slot lies inside this launch's tile
                   const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
@@ -620,7 +637,8 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   }
   const int grid = (int)(items < c.num_sms ? items : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  const bool plain = ks == 1 && p.thr == nullptr && p.row_slot == nullptr && a.kv.page_size == 0;
+  const bool plain =
+      ks == 1 && p.thr == nullptr && p.row_slot == nullptr && a.kv.page_size == 0 && a.kv.seqlens == nullptr;
   auto kern = plain ? indexer_tc_kernel<DI, HI, true> : indexer_tc_kernel<DI, HI, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;

@@ -36,9 +36,8 @@
 // TMEM accumulator is rescaled once (each softmax warp its half of the value
 // columns), after the previous P V has landed.
 //
-// Warp roles (512 threads): warp 0 owns TMEM and issues Q K^T of the even
-// chunks, warp 15 Q K^T of the odd chunks and every P V (one thread issuing
-// N = 64 MMAs back to back cannot keep the tensor pipe busy), warps 1-3 and
+// Warp roles (480 threads): warp 0 owns TMEM and issues the MMAs (whichever
+// is ready: Q K^T of the next chunk or P V of the oldest), warps 1-3 and
 // 12-14 gather, warps 4-11 run the softmax (thread = head row) and write the
 // output.  Decode splits the selected keys of each query over several CTAs
 // and merges the partial results with a combine kernel.  Every barrier that
@@ -65,12 +64,7 @@ constexpr int kSBuf = 2;        // S/P buffers in TMEM
 constexpr int kMmaWarp = 0, kFirstSoftmaxWarp = 4, kSoftmaxWarps = 8;
 constexpr int kGatherPerSlot = 3;
 constexpr int kFirstGatherB = kFirstSoftmaxWarp + kSoftmaxWarps;
-// A second MMA-issuing warp: one thread issuing back-to-back N = 64 MMAs
-// cannot keep the tensor pipe busy, so warp 0 issues Q K^T of the even
-// chunks and this warp Q K^T of the odd chunks and every P V (P V stays with
-// one thread: its accumulation into O must keep chunk order).
-constexpr int kMmaWarp2 = kFirstGatherB + kGatherPerSlot;
-constexpr int kThreads = 32 * (kMmaWarp2 + 1);
+constexpr int kThreads = 32 * (kFirstGatherB + kGatherPerSlot);
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -203,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], kSoftmaxWarps);
       mbar_init(&pv_done[i], 1);
     }
-    mbar_init(mma_done, 2);   // one commit from each MMA-issuing warp
+    mbar_init(mma_done, 1);
     for (int i = 0; i < kSBuf * 4 + 4; ++i) mbar_init(&mx_bar[i], 2);
     *abort_flag = 0;
     fence_mbar_init();
@@ -229,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return __all_sync(0xffffffffu, r);
   };
 
-  if (warp != kMmaWarp && warp != kMmaWarp2 && (warp < kFirstSoftmaxWarp || warp >= kFirstGatherB)) {
+  if (warp != kMmaWarp && (warp < kFirstSoftmaxWarp || warp >= kFirstGatherB)) {
     // ------------------------------------------------------------ gather
     // slot half h of every chunk; warp g of the half copies atoms g, g+3, g+6
     const int h = warp < kFirstSoftmaxWarp ? 0 : 1;
@@ -244,6 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int c16 = lane & 7, rg = lane >> 3;  // 16-byte column chunk, row group
     const int32_t* irow = dense ? nullptr : p.idx + (size_t)row * p.k;
+    // the sequence's rows of a contiguous cache; in the paged form, the cache
+    // row of its key 0 (every sequence has at least T keys), which empty
+    // slots copy (pool row 0 if that page is unmapped)
+    const uint16_t* kvb = p.kv + (size_t)b * p.S * DK;
+    long long row0 = PAGED && nchunks > 0 ? p.map.row<true>(b, 0) : 0;
+    if (row0 < 0) row0 = 0;
     // indices of this half of chunk j, loaded one chunk ahead
     int ivn[kSlotKeys / 4];
     auto load_idx = [&](int j) {
@@ -270,31 +270,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
           v = -1;
         }
-        long long cr = v >= 0 ? p.map.row<PAGED>(b, v) : -1;   // cache row of key v
-        if (v >= 0 && cr < 0) {
-          if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
-          v = -1;
+        // cache row of key v: a page lookup in the paged form (an unmapped
+        // page is reported and the slot emptied); the contiguous form keeps
+        // the row arithmetic out of this loop
+        long long cr = 0;
+        if constexpr (PAGED) {
+          cr = v >= 0 ? p.map.row<true>(b, v) : -1;
+          if (v >= 0 && cr < 0) {
+            if (c16 == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
+            v = -1;
+          }
         }
         const bool valid = v >= 0;
         // lanes 0, 8, 16, 24 hold rows 4m .. 4m+3
         const uint32_t bal = __ballot_sync(0xffffffffu, valid);
         mask |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u)) << (4 * m);
-        // an empty or invalid slot is zero-filled (a copy that reads 0
-        // bytes), so that no stale or non-finite shared memory meets its zero
-        // probability in P V
-        const size_t crow = (size_t)(valid ? cr : 0);
-        const uint32_t nbytes = valid ? 16u : 0u;
-        const uint16_t* src = p.kv + crow * DK;
+        // an empty or invalid slot copies the sequence's first key row (a
+        // finite row of the caller's cache), which then meets probability 0
+        // in P V
+        const size_t crow = PAGED ? (size_t)(valid ? cr : row0) : (size_t)b * p.S + (valid ? v : 0);
+        const uint16_t* src = PAGED ? p.kv + crow * DK : kvb + (size_t)(valid ? v : 0) * DK;
 #pragma unroll
-        for (int a0 = 0; a0 < C::ATOMS; a0 += kGatherPerSlot) {
+        for (int a0 = 0; a0 < C::NATOM; a0 += kGatherPerSlot) {
           const int a = a0 + g;
-          uint8_t* dst = slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4);
-          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2) {
-            cp_async16_zfill(dst, src + a * 64 + c16 * 8, nbytes);
-          } else if (SEPV && a >= C::NATOM && a < C::ATOMS) {
-            // value atom: columns half * DVH + (a - NATOM) * 64 .. of the value row
-            const int vc = (a - C::NATOM) * 64 + c16 * 8;
-            if (vc < C::DVH) cp_async16_zfill(dst, p.v + crow * DV + half * C::DVH + vc, nbytes);
+          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2)
+            cp_async16(slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
+        }
+        if constexpr (SEPV) {
+          // this CTA's value columns [half * DVH, (half + 1) * DVH) of the
+          // value row, in atoms NATOM, NATOM + 1, ...
+          const uint16_t* vsrc = p.v + crow * DV + half * C::DVH;
+#pragma unroll
+          for (int va0 = 0; va0 < C::NVATOM; va0 += kGatherPerSlot) {
+            const int va = va0 + g;
+            if (va < C::NVATOM && va * 64 + c16 * 8 < C::DVH)
+              cp_async16(slotp + (C::NATOM + va) * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4),
+                         vsrc + va * 64 + c16 * 8);
           }
         }
       }
@@ -308,13 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait<0>();
     // drain: the Q load must have landed before this CTA's memory is reused
     if (q_issued) mbar_wait(q_full, 0, p.wait_ns, no_abort);
-  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
-    // warp 0: Q K^T of even chunks; warp kMmaWarp2: Q K^T of odd chunks and
-    // all P V.  Chunk j uses S buffer j % 2 and ring slots 2 (j % NCH), +1.
+    // chunk j uses S buffer j % 2 and ring slots 2 (j % NCH), 2 (j % NCH) + 1
     if (lane == 0) {
-      const int qk_par = warp == kMmaWarp ? 0 : 1;
-      const bool does_pv = warp == kMmaWarp2;
       constexpr uint32_t idesc_qk = make_idesc(kFmtBF16, kFmtBF16, 0, 0, 128, kN);
       constexpr uint32_t idesc_pv = make_idesc(kFmtBF16, kFmtBF16, 0, 1, 128, C::DVH);
       // descriptors are built once; a step only adds its byte offset >> 4 to
@@ -327,12 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = nchunks == 0 || ((C::QS_ATOMS == 0 || mbar_wait(q_full, 0, p.wait_ns, ab)) &&
                                  mbar_wait(q_ready, 0, p.wait_ns, ab));
       if (!ok) fail(3);
-      // Issue whichever MMA of this thread is ready: Q K^T of chunk qk once
-      // its rows have landed and P V of chunk qk - kSBuf has freed its S
-      // buffer; P V of chunk pv once its probabilities are written (which
-      // implies Q K^T of pv has completed, whichever thread issued it).
-      int qk = qk_par, pv = 0;
-      int last_qk = -1;
+      // Issue whichever MMA is ready: Q K^T of chunk qk once its rows have
+      // landed and P V of chunk qk - kSBuf has freed its S buffer; P V of
+      // chunk pv once its probabilities are written.
+      int qk = 0, pv = 0;
       // P V of chunk pv: 4 K steps of 16 keys, A = P (TMEM), B = V (MN-major);
       // its commits free the chunk's S buffer and both ring slots
       auto issue_pv = [&]() {
@@ -365,9 +371,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       uint64_t t_idle = 0;
       uint32_t spins = 0;
-      while (ok && (qk < nchunks || (does_pv && pv < nchunks))) {
+      while (ok && pv < nchunks) {
         bool progressed = false;
-        if (qk < nchunks) {
+        if (qk < nchunks && qk < pv + kSBuf) {
           const int s0 = (2 * qk) % kSlots, sb = qk % kSBuf;
           const uint32_t par = (uint32_t)((2 * qk) / kSlots) & 1;
           if (mbar_test_wait(&kv_full[s0], par) && mbar_test_wait(&kv_full[s0 + 1], par) &&
@@ -389,12 +395,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             mma_commit(&s_full[sb]);
-            last_qk = qk;
-            qk += 2;
+            ++qk;
             progressed = true;
           }
         }
-        if (does_pv && pv < nchunks && mbar_test_wait(&p_full[pv % kSBuf], (pv / kSBuf) & 1)) {
+        if (pv < qk && mbar_test_wait(&p_full[pv % kSBuf], (pv / kSBuf) & 1)) {
           issue_pv();
           progressed = true;
         }
@@ -404,9 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // nothing ready: doze briefly on the event most likely next, with
         // bounded idle time, and abort when another role failed
-        if (does_pv && pv < nchunks && (qk >= nchunks || pv < qk))
+        if (pv < qk)
           mbar_try_wait_hint(&p_full[pv % kSBuf], (pv / kSBuf) & 1, 200);
-        else if (qk < nchunks)
+        else
           mbar_try_wait_hint(&kv_full[(2 * qk) % kSlots], (uint32_t)((2 * qk) / kSlots) & 1, 200);
         if (++spins == 1) t_idle = global_ns();
         if ((spins & 1023u) == 0u) {
@@ -418,19 +423,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // both issuers commit once: the phase completes when every MMA of
-      // both has finished
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
       // drain: the last arrivals of each commit barrier are not always waited
       // by their consumers; make sure they have landed before the CTA exits
-      if (does_pv) {
-        for (int c = max(0, 2 * pv - kSlots); c < 2 * pv; ++c)
-          mbar_wait(&kv_empty[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
-        for (int i = max(0, pv - kSBuf); i < pv; ++i)
-          mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
-      }
-      if (last_qk >= 0) mbar_wait(&s_full[last_qk % kSBuf], (last_qk / kSBuf) & 1, p.wait_ns, no_abort);
+      for (int c = max(0, 2 * pv - kSlots); c < 2 * pv; ++c)
+        mbar_wait(&kv_empty[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
+      for (int i = max(0, pv - kSBuf); i < pv; ++i)
+        mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
+      for (int i = max(0, qk - kSBuf); i < qk; ++i)
+        mbar_wait(&s_full[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
