@@ -13,9 +13,12 @@ by replay (per-kernel times from one graph per launch group), falling back
 to eager steps if the capture fails or its selection differs.
 
 Kernel timing: each step calls the C-ABI step entry points in the order
-dsa_forward uses, with CUDA events between launches on the launching stream,
-so every kernel's share of the step is measured live; `e2e` runs dsa_forward
-itself on host (pinned) buffers with the copies inside the timed region.
+dsa_forward uses with a full workspace, with CUDA events between launches on
+the launching stream, so every kernel's share of the step is measured live;
+`e2e` runs dsa_forward itself on host (pinned) buffers with the copies inside
+the timed region.  `alternatives.select_fused` times dsa_select over the same
+query blocks on its own (the fused indexer + top-k that dsa_forward takes when
+its workspace has no room for the score tile); it is not part of the step.
 
 Inputs are synthetic (long_context_05_b200.inputs), larger than L2 for the
 prefill; L2 is flushed between timed steps anyway (a 256 MiB write outside
@@ -215,18 +218,17 @@ class DsaRunner:
         self.ws = dsa.alloc_workspace(self.shape)
         self.outs = dsa.alloc_outputs(wl)
         self.ld = (wl.S + 63) // 64 * 64
-        if wl.decode:
-            # decode scores its rows into the workspace's score tile; the
-            # top-k's scratch (histograms of the split path for few long
-            # rows) follows it, 256-byte aligned, as in dsa_forward
-            nscore = wl.B * self.rows_per_block() * self.ld * 4
-            self.scores = self.ws[:nscore].view(torch.float32).view(-1, self.ld)
-            self.topk_ws = self.ws[(nscore + 255) // 256 * 256:]
-        else:
-            # prefill selects through dsa_select (its own use of the
-            # workspace); the index fill of the dense rows reads no score
-            self.scores = torch.zeros(1, self.ld, dtype=torch.float32, device="cuda")
-            self.topk_ws = None
+        # each query block scores its rows into the workspace's score tile;
+        # the top-k's scratch (histograms of the split path for few long rows,
+        # as in decode) follows it, 256-byte aligned, as in dsa_forward
+        nscore = wl.B * self.rows_per_block() * self.ld * 4
+        self.scores = self.ws[:nscore].view(torch.float32).view(-1, self.ld)
+        self.topk_ws = self.ws[(nscore + 255) // 256 * 256:] if wl.decode else None
+        # the fused selection (dsa_select) where it applies: its own, smaller
+        # workspace; timed beside the step as the alternative to indexer + topk
+        self.ws_fused = None
+        if not wl.decode and dsa.select_workspace_size(self.shape) < dsa.workspace_size(self.shape):
+            self.ws_fused = dsa.alloc_workspace(self.shape, fused=True)
         self.stream = torch.cuda.current_stream()
 
     def rows_per_block(self):
@@ -247,25 +249,15 @@ class DsaRunner:
             return e
 
         dr = dense_rows(wl)
-        sel = "select" if not wl.decode else "topk"
         if dr:
             # rows that keep all their visible keys: the index fill only
             e0 = mark()
             d.topk(self.shape, self.scores, 0, dr, o.idx, self.topk_ws)
             e1 = mark()
             if ev is not None:
-                ev.append((sel, e0, e1))
+                ev.append(("topk", e0, e1))
         for q0 in range(dr, wl.T, qb):
             cnt = min(qb, wl.T - q0)
-            if not wl.decode:
-                # prefill: steps A and B of the block in one call (no score
-                # tile over long contexts)
-                e0 = mark()
-                d.select(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, o.idx, self.ws)
-                e1 = mark()
-                if ev is not None:
-                    ev.append(("select", e0, e1))
-                continue
             e0 = mark()
             d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, self.scores)
             e1 = mark()
@@ -281,7 +273,8 @@ class DsaRunner:
             ev.append(("sparse_attn", e3, e4))
 
     def step_part(self, name):
-        """One of the step's launch groups alone (indexer, topk or sparse_attn)."""
+        """One of the step's launch groups alone (indexer, topk or sparse_attn),
+        or "select": steps A and B of every block through the fused selection."""
         d, wl, i, o = self.dsa, self.wl, self.inp, self.outs
         qb = self.rows_per_block()
         if name == "sparse_attn":
@@ -293,7 +286,8 @@ class DsaRunner:
         for q0 in range(dr, wl.T, qb):
             cnt = min(qb, wl.T - q0)
             if name == "select":
-                d.select(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, o.idx, self.ws)
+                d.select(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, o.idx,
+                         self.ws_fused)
             elif name == "indexer":
                 d.indexer_scores(self.shape, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt,
                                  self.scores)
@@ -336,6 +330,33 @@ def time_steps(runner, steps, warmup, ws):
     if st != 0:
         raise RuntimeError(f"device error {st} detail {det:#x}")
     return total_ms, per_kernel, launches
+
+
+def time_part(runner, name, steps, warmup, ws):
+    """Device time per step of one launch group run alone (flushed L2, same
+    barriers as time_steps), in ms, max over ranks."""
+    flush = Flusher()
+    for _ in range(warmup):
+        runner.step_part(name)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        runner.step_part(name)
+        b.record()
+        b.synchronize()
+        total += a.elapsed_time(b)
+    torch.cuda.synchronize()
+    barrier(ws)
+    st, det = runner.dsa.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {det:#x}")
+    return max_over_ranks(total / steps, ws)
 
 
 def capture_step_graphs(runner, warmup):
@@ -537,6 +558,11 @@ def gpu_arm(args):
     clocks.start()
     total_ms, per_kernel, launches = time_steps(runner, args.steps, args.warmup, ws)
     ms_step = max_over_ranks(total_ms / args.steps, ws)
+    # the fused selection, timed alone over the same blocks (every rank takes
+    # the same branch: the workload is the same on all)
+    fused_ms = None
+    if runner.ws_fused is not None:
+        fused_ms = time_part(runner, "select", args.steps, min(args.warmup, 1), ws)
     dec = None
     if wl_dec is not None:
         drun = DsaRunner(wl_dec, seed_offset=rank)
@@ -584,6 +610,16 @@ def gpu_arm(args):
 
     rep = kernel_report(runner.wl, per_kernel, args.steps, peaks, peak_src, sustained=True)
     top = max(rep.items(), key=lambda kv: kv[1]["ms_per_step"])
+    alternatives = None
+    if fused_ms is not None:
+        f = kernel_report(runner.wl, {"select": [fused_ms] * args.steps}, args.steps, peaks, peak_src,
+                          sustained=True)["select"]
+        f.pop("share", None)
+        sel_ms = sum(rep[n]["ms_per_step"] for n in ("indexer", "topk") if n in rep)
+        f["vs_indexer_topk"] = fused_ms / sel_ms if sel_ms > 0 else None
+        f["workspace_bytes"] = int(runner.ws_fused.numel())
+        f["score_tile_workspace_bytes"] = int(runner.ws.numel())
+        alternatives = {"select_fused": f}
     tokens = ws * wl.B * wl.T
     line = {
         "metric": METRIC,
@@ -607,6 +643,7 @@ def gpu_arm(args):
                      "traffic": measured_traffic(wl.name, top[0]),
                      "peak_note": top[1]["peak_note"]},
         "kernels": rep,
+        "alternatives": alternatives,
         "decode": dec,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -137,8 +137,17 @@ DSA_API int dsa_version(void);
 DSA_API const char* dsa_status_string(dsa_status status);
 
 /* Bytes of workspace dsa_forward / dsa_prefill / dsa_decode need for `shape`
- * (it covers dsa_topk and dsa_sparse_attn too).  0 if the shape is invalid. */
+ * with the query block's FP32 score tile held in it (it covers dsa_topk,
+ * dsa_select and dsa_sparse_attn too).  0 if the shape is invalid. */
 DSA_API size_t dsa_workspace_size(const dsa_shape* shape);
+
+/* Bytes of workspace for dsa_select, and the least a prefill dsa_forward
+ * accepts, where the fused selection applies (prefill, contiguous caches,
+ * S >= 32768, S a multiple of 16): its regions replace the score tile, about
+ * a third of the tile's size (0.64 GiB instead of 2 GiB for a 4096-row block
+ * of a 128K context).  Elsewhere equal to dsa_workspace_size.  0 if the shape
+ * is invalid. */
+DSA_API size_t dsa_select_workspace_size(const dsa_shape* shape);
 
 /* Step A -- lightning indexer scores for queries [q_begin, q_begin + q_count)
  * of every sequence.  scores row (b * q_count + i) holds query
@@ -172,7 +181,7 @@ DSA_API dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
 
 /* Steps A and B together for queries [q_begin, q_begin + q_count): writes the
  * selection idx[b, t, 0..k) as dsa_topk does (ties to the lower index, -1
- * after the last).  ws: dsa_workspace_size(shape) bytes.
+ * after the last).  ws: dsa_select_workspace_size(shape) bytes.
  * In prefill over long contexts (S >= 32768, S a multiple of 16, contiguous
  * caches) the query block's score matrix is never stored (the pages ask that
  * the selection be cache-aware and stay on the device: sider.ai blog on
@@ -251,7 +260,12 @@ DSA_API dsa_status dsa_dense_attn(const dsa_shape* shape, const uint16_t* q,
  * up to S) skip steps A and B: their selection is all visible keys, written
  * to idx_out as 0..pos(t), and step C runs on them densely.
  * idx_out: [B, T, k] int32 receives the selection (required).
- * ws: at least dsa_workspace_size(shape) bytes. */
+ * ws: dsa_workspace_size(shape) bytes, or in prefill at least
+ * dsa_select_workspace_size(shape): a workspace that holds the score tile
+ * runs steps A and B as dsa_indexer_scores + dsa_topk; a smaller one that
+ * holds the fused selection's regions runs them as dsa_select does (same
+ * selection, less memory, more time); anything smaller is
+ * DSA_ERR_WORKSPACE. */
 DSA_API dsa_status dsa_forward(const dsa_shape* shape, const dsa_inputs* in,
                        uint16_t* out, float* lse, int32_t* idx_out, void* ws,
                        size_t ws_bytes, void* stream);

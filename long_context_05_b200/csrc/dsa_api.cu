@@ -133,7 +133,9 @@ constexpr int kTargetNum = 3, kTargetDen = 2;   // about 1.5 k candidates expect
 constexpr int kRowCap = 6144;     // candidates a row's list holds (<= the top-k's shared capacity)
 constexpr int kWarpSlack = 2;     // warp lists hold twice the expected candidates
 
-bool fused_select(const dsa_shape* s) {
+// The fused selection applies: prefill over a contiguous cache long enough
+// for the key sample to leave few candidates per row.
+bool fused_select_ok(const dsa_shape* s) {
   return s->mode == DSA_PREFILL && s->page_size == 0 && s->S % kSampleStride == 0 &&
          s->S >= 4 * topk_cand_cap();
 }
@@ -162,11 +164,13 @@ struct WsLayout {
   int q_rows;
 };
 
-WsLayout ws_layout(const dsa_shape* s, int num_sms) {
+// fused: the fused selection's regions in place of the score tile (only
+// where fused_select_ok holds)
+WsLayout ws_layout(const dsa_shape* s, int num_sms, bool fused) {
   WsLayout L;
   L.q_rows = s->mode == DSA_DECODE ? s->T : q_block_of(s);
   L.scores_off = 0;
-  L.fused = fused_select(s);
+  L.fused = fused && fused_select_ok(s);
   L.cap = kRowCap < topk_cand_cap() ? kRowCap : topk_cand_cap();
   L.ld_s = (int64_t)round_up((size_t)(s->S / kSampleStride), 64);
   if (L.fused) {
@@ -214,6 +218,16 @@ WsLayout ws_layout(const dsa_shape* s, int num_sms) {
   L.topk_bytes = topk_uses_workspace(topk_rows, s->S, num_sms) ? round_up(topk_workspace_bytes(topk_rows), 256) : 0;
   L.total = L.topk_off + L.topk_bytes;
   return L;
+}
+
+// The layout a call given ws_bytes of workspace takes: the score tile when
+// it fits, else the fused selection's regions when they fit, else the score
+// tile's (which the caller then reports as too small).
+WsLayout ws_choose(const dsa_shape* s, int num_sms, size_t ws_bytes) {
+  WsLayout L = ws_layout(s, num_sms, false);
+  if (ws_bytes >= L.total || !fused_select_ok(s)) return L;
+  WsLayout F = ws_layout(s, num_sms, true);
+  return ws_bytes >= F.total ? F : L;
 }
 
 dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
@@ -392,7 +406,16 @@ size_t dsa_workspace_size(const dsa_shape* s) {
   int dev = 0;
   int sms = 148;
   if (device_info(&d, &dev) == DSA_OK) sms = d.num_sms;
-  return ws_layout(s, sms).total;
+  return ws_layout(s, sms, false).total;
+}
+
+size_t dsa_select_workspace_size(const dsa_shape* s) {
+  if (check_shape(s) != DSA_OK) return 0;
+  DeviceInfo d;
+  int dev = 0;
+  int sms = 148;
+  if (device_info(&d, &dev) == DSA_OK) sms = d.num_sms;
+  return ws_layout(s, sms, true).total;
 }
 
 dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_I, const float* q_scale, const float* w,
@@ -430,7 +453,7 @@ dsa_status dsa_select(const dsa_shape* s, const uint8_t* q_I, const float* q_sca
   if (q_begin < 0 || q_count < 0 || q_begin + q_count > s->T) return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
-  WsLayout L = ws_layout(s, c.num_sms);
+  WsLayout L = ws_layout(s, c.num_sms, true);
   if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
   for (int q0 = q_begin; q0 < q_begin + q_count; q0 += L.q_rows) {
     const int cnt = (q_begin + q_count - q0) < L.q_rows ? (q_begin + q_count - q0) : L.q_rows;
@@ -447,7 +470,7 @@ dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t
     return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
-  WsLayout L = ws_layout(s, c.num_sms);
+  WsLayout L = ws_layout(s, c.num_sms, false);
   float* part = nullptr;
   if (L.nsplit > 1 || (s->mode == DSA_DECODE && attn_decode_nsplit(s->k) > 1)) {
     if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
@@ -464,7 +487,7 @@ dsa_status dsa_dense_attn(const dsa_shape* s, const uint16_t* q, const uint16_t*
     return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
-  WsLayout L = ws_layout(s, c.num_sms);
+  WsLayout L = ws_layout(s, c.num_sms, false);
   float* part = nullptr;
   if (L.nsplit_dense > 1) {
     if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
@@ -483,7 +506,7 @@ dsa_status dsa_forward(const dsa_shape* s, const dsa_inputs* in, uint16_t* out, 
     return DSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, &c)) != DSA_OK) return st;
-  WsLayout L = ws_layout(s, c.num_sms);
+  WsLayout L = ws_choose(s, c.num_sms, ws == nullptr ? 0 : ws_bytes);
   if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + L.scores_off);
   float* part = L.part_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) + L.part_off) : nullptr;

@@ -25,7 +25,8 @@ STATUS = {
 }
 
 EXPORTS = [
-    "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk",
+    "dsa_version", "dsa_status_string", "dsa_workspace_size", "dsa_select_workspace_size", "dsa_indexer_scores",
+    "dsa_topk",
     "dsa_sparse_attn", "dsa_forward", "dsa_prefill", "dsa_decode", "dsa_get_device_error",
     "dsa_set_wait_timeout_us", "dsa_launch_count", "dsa_selftest_wait_timeout", "dsa_topk_static",
     "dsa_dense_attn", "dsa_topk_candidates", "dsa_topk_merge", "dsa_attn_combine", "dsa_select",
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_status_string.argtypes = [i]
         L.dsa_workspace_size.restype = sz
         L.dsa_workspace_size.argtypes = [sp]
+        L.dsa_select_workspace_size.restype = sz
+        L.dsa_select_workspace_size.argtypes = [sp]
         L.dsa_indexer_scores.restype = i
         L.dsa_indexer_scores.argtypes = [sp, vp, vp, vp, vp, vp, i, i, vp, i64, vp]
         L.dsa_topk.restype = i
@@ -172,10 +175,16 @@ def workspace_size(shape: Shape) -> int:
     return int(lib().dsa_workspace_size(ctypes.byref(shape)))
 
 
-def alloc_workspace(shape: Shape) -> torch.Tensor:
-    n = workspace_size(shape)
+def select_workspace_size(shape: Shape) -> int:
+    return int(lib().dsa_select_workspace_size(ctypes.byref(shape)))
+
+
+def alloc_workspace(shape: Shape, fused: bool = False) -> torch.Tensor:
+    """dsa_workspace_size bytes, or with fused=True dsa_select_workspace_size
+    (dsa_select's size; a prefill forward given it takes the fused selection)."""
+    n = select_workspace_size(shape) if fused else workspace_size(shape)
     if n == 0:
-        raise DsaError("dsa_workspace_size", 1)
+        raise DsaError("dsa_select_workspace_size" if fused else "dsa_workspace_size", 1)
     return torch.empty(n, dtype=torch.uint8, device="cuda")
 
 

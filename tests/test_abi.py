@@ -62,6 +62,18 @@ def test_host_side_calls_without_gpu(libpath):
     assert dsa.workspace_size(dsa.make_shape(None, **paged, page_size=64, pages_per_seq=15, num_pages=40,
                                              block_table=fake_table)) == 0      # 15 * 64 < S
     assert dsa.workspace_size(dsa.make_shape(None, **paged, page_size=64, pages_per_seq=16, num_pages=40)) == 0
+    # the fused selection's workspace: about a third of the 4096 x 131072 FP32
+    # score tile (2 GiB) for a 128K prefill block; the score tile's size where
+    # the fused selection does not apply (decode, short contexts)
+    from long_context_05_b200.inputs import WORKLOADS
+    big = dsa.make_shape(WORKLOADS["prefill_128k"])
+    tile = 4096 * 131072 * 4
+    assert dsa.workspace_size(big) >= tile
+    assert 0 < dsa.select_workspace_size(big) < tile // 3
+    for name in ("decode_128k_b8", "prefill_8k"):
+        sh = dsa.make_shape(WORKLOADS[name])
+        assert dsa.select_workspace_size(sh) == dsa.workspace_size(sh) > 0
+    assert dsa.select_workspace_size(bad) == 0
     assert L.dsa_launch_count() == 0
 
 

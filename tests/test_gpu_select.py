@@ -40,7 +40,7 @@ def _materialised(wl, inp, shape, q0, cnt):
 def _fused(wl, inp, shape, q0, cnt):
     idx = torch.full((wl.B, wl.T, wl.k), -9, dtype=torch.int32, device="cuda")
     dsa.select(shape, inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], q0, cnt, idx,
-               dsa.alloc_workspace(shape))
+               dsa.alloc_workspace(shape, fused=True))
     st, det = dsa.device_error()
     assert st == 0, (st, hex(det))
     return idx
@@ -71,14 +71,26 @@ def test_fused_selection_equals_materialised_128k_rows():
         P.check_selection(g[t], idx_o, sc, False, f"fused t={t}")
 
 
-def test_fused_workspace_is_smaller_than_the_score_tile():
-    """The 128K prefill's workspace no longer holds a 4096 x 131072 FP32
-    score tile (2 GiB): the key sample, the candidate lists and the repair
-    tile take about 0.64 GiB."""
-    wl = WORKLOADS["prefill_128k"]
-    n = dsa.workspace_size(dsa.make_shape(wl))
-    tile = wl.q_block * wl.S * 4                          # 2 GiB
-    assert n < tile // 3, n
+def test_forward_takes_the_fused_selection_in_a_small_workspace():
+    """dsa_forward given dsa_select_workspace_size bytes (no room for the
+    score tile) selects through the fused path: the same selection and the
+    same output as with the full workspace."""
+    wl = WORKLOADS["prefill_chunk_128k"]
+    inp = make_inputs(wl, "cuda")
+    inp.pop("needle_pos", None)
+    shape = dsa.make_shape(wl)
+    small, full = dsa.alloc_workspace(shape, fused=True), dsa.alloc_workspace(shape)
+    assert small.numel() < full.numel() // 2        # 108 MiB instead of the 256 MiB score tile
+    a, b = dsa.alloc_outputs(wl), dsa.alloc_outputs(wl)
+    dsa.forward(shape, inp, a.out, a.lse, a.idx, small)
+    dsa.forward(shape, inp, b.out, b.lse, b.idx, full)
+    st, det = dsa.device_error()
+    assert st == 0, (st, hex(det))
+    _same_sets(a.idx, b.idx, range(wl.T))
+    # the same sets in another slot order: outputs agree to FP32 summation order
+    assert torch.allclose(a.out.float(), b.out.float(), atol=2e-2, rtol=2e-2)
+    with pytest.raises(dsa.DsaError):
+        dsa.forward(shape, inp, a.out, a.lse, a.idx, small[: small.numel() - 256])
 
 
 def test_fused_selection_block_of_128k_prefill():
