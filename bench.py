@@ -52,14 +52,16 @@ PREFILL = "prefill_128k"
 DECODE = "decode_128k_b8"
 
 # DRAM bytes (read + write) of one sparse-attention launch on prefill_128k,
-# from one ncu capture of the full-size launch (dram__bytes_read.sum 21.73 GB
-# + dram__bytes_write.sum 17.21 GB, one pass; the command is kept with the
-# capture summaries under profiles/).  It holds only for the kernel
-# source it was taken from, so the bench reports it only while that source's
-# hash matches.
-ATTN_TRAFFIC = {"workload": "prefill_128k", "kernel": "sparse_attn", "bytes": 21.73e9 + 17.21e9,
+# scaled from an ncu capture of the same kernel on prefill_chunk_128k (the
+# command is kept with the capture summaries under profiles/).  It holds only
+# for the kernel source it was taken from, so the bench reports it only while
+# that source's hash matches.
+ATTN_TRAFFIC = {"workload": "prefill_128k", "kernel": "sparse_attn",
+                # DRAM read + write of one prefill_chunk_128k launch (92.37 MB +
+                # 32.00 MB, ncu) times 256, the ratio of query rows
+                "bytes": 92.37e6 * 256 + 32.00e6 * 256,
                 "source": "long_context_05_b200/csrc/sparse_attn.cu",
-                "sha256": "2b5a5b965a6d2f00e8b2f2543ee7af060875d29cc3825ee0cf633465863c0aed"}
+                "sha256": "1014d28eb4e008b7b4ad86ac641c8086294879e2df7ff9a8abf6871d01a86f78"}
 
 
 def measured_traffic(workload: str, kernel: str):
