@@ -448,10 +448,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the splits of each (row, head): 64 threads per (row, head), eight
-// value columns each (one 16-byte load of FP16 per split).
+// value columns each (one 16-byte load of FP16 per split).  The splits are
+// taken 16 at a time with every load of a batch issued before the first is
+// used, so a thread waits for memory once per batch, not once per split.
 __global__ void __launch_bounds__(256) attn_combine_f16_kernel(const __half* part_o, const float* part_lse,
                                                                uint16_t* out, float* lse, int rows, int H,
                                                                int nsplit) {
+  constexpr int kBatch = 16;
   // results of the attention grid are visible after this
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long gh = (long long)blockIdx.x * 4 + (threadIdx.x >> 6);
@@ -459,6 +462,7 @@ __global__ void __launch_bounds__(256) attn_combine_f16_kernel(const __half* par
   const int row = (int)(gh / H), h = (int)(gh - (long long)(gh / H) * H);
   const int d0 = (threadIdx.x & 63) * 8;
   const float* ls = part_lse + (size_t)row * nsplit * H + h;
+  const __half* po = part_o + ((size_t)row * nsplit * H + h) * DV + d0;   // split s at + s * H * DV
   float mx = -INFINITY;
   for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, ls[(size_t)s * H]);
   float acc[8];
@@ -466,18 +470,27 @@ __global__ void __launch_bounds__(256) attn_combine_f16_kernel(const __half* par
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   float wsum = 0.f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float l = ls[(size_t)s * H];
-      if (l == -INFINITY) continue;
-      const float w = exp2f(l - mx);
-      wsum += w;
-      const uint4 v = *reinterpret_cast<const uint4*>(part_o + (((size_t)row * nsplit + s) * H + h) * DV + d0);
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
+      float w[kBatch];
+      uint4 v[kBatch];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-        acc[2 * i] = fmaf(w, f.x, acc[2 * i]);
-        acc[2 * i + 1] = fmaf(w, f.y, acc[2 * i + 1]);
+      for (int i = 0; i < kBatch; ++i) {
+        const int s = s0 + i;
+        const float l = s < nsplit ? ls[(size_t)s * H] : -INFINITY;
+        w[i] = l == -INFINITY ? 0.f : exp2f(l - mx);
+        v[i] = l == -INFINITY ? make_uint4(0u, 0u, 0u, 0u)
+                              : *reinterpret_cast<const uint4*>(po + (size_t)s * H * DV);
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        wsum += w[i];
+        const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[c]));
+          acc[2 * c] = fmaf(w[i], f.x, acc[2 * c]);
+          acc[2 * c + 1] = fmaf(w[i], f.y, acc[2 * c + 1]);
+        }
       }
     }
   }
