@@ -200,6 +200,9 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // a programmatically dependent kernel (the decode top-k) may be scheduled
+  // now; it waits for this grid's scores before reading them
+  pdl_launch_dependents();
   // With at most half of the B sub-tiles in use (few queries per item, as in
   // decode), the B region holds two item buffers, so the next item's B and
   // its first key tiles load while the current item's MMAs run.

@@ -147,6 +147,25 @@ struct AttnArgs {
 // counts every kernel launch (dsa_launch_count)
 void note_launches(int n);
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the one before it on the stream finishes, and must call pdl_wait
+// (sm100.cuh) before it reads anything that kernel writes.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 cudaError_t launch_indexer(const LaunchCtx& c, const IndexerArgs& a);
 // ws: optional scratch for the split path (few long rows); see topk.cu
 cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t ws_bytes);

@@ -330,6 +330,18 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------------------------ launch order
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start once every CTA of the kernel before it has called
+// pdl_launch_dependents (or exited); pdl_wait then blocks until that kernel
+// has completed and its memory is visible.  Both return at once in a kernel
+// launched the ordinary way.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ misc
 
 // 2^x with the hardware approximation (flushes subnormal results to zero)

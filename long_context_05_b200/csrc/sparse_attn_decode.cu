@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   // the combine kernel may be scheduled now; it waits for this grid's results
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_launch_dependents();
   uint8_t* sQ = smem + OFF_Q;
   uint8_t* sKV = smem + OFF_KV;
   uint64_t* sMask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
@@ -181,6 +181,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sQ + a * kQAtomBytes, &tm_q, q_full, kQT + a * 64, row * p.H);
       q_issued = true;
     }
+    // the selection is the kernel before this one's output (this kernel is
+    // its programmatic dependent: barrier set-up, TMEM allocation and the Q
+    // loads above overlap its tail)
+    pdl_wait();
     // the 64 indices of this half: lane l holds slots l and l + 32
     int iv2[2];
 #pragma unroll
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(256) attn_combine_f16_kernel(const __half* par
                                                                int nsplit) {
   constexpr int kBatch = 16;
   // results of the attention grid are visible after this
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   const long long gh = (long long)blockIdx.x * 4 + (threadIdx.x >> 6);
   if (gh >= (long long)rows * H) return;
   const int row = (int)(gh / H), h = (int)(gh - (long long)(gh / H) * H);
@@ -548,7 +552,10 @@ cudaError_t launch_sparse_attn_decode(const LaunchCtx& c, const AttnArgs& a, voi
   auto kern = a.map.page_size != 0 ? sparse_attn_decode_kernel<true> : sparse_attn_decode_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(rows * p.nsplit), kThreads, kSmem, c.stream>>>(tm_q, p);
+  // a programmatic dependent of the top-k: its prologue overlaps the
+  // selection's last launch, which runs only one block per row
+  e = launch_pdl(kern, dim3((unsigned)(rows * p.nsplit)), dim3(kThreads), kSmem, c.stream, tm_q, p);
+  if (e != cudaSuccess) return e;
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.nsplit == 1) return e;

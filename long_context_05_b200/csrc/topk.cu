@@ -33,9 +33,13 @@
 // counts, then one global atomic per list and block); one block per row
 // finishes step 3 on that list.
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace dsa {
 namespace {
+
+using sm100::pdl_launch_dependents;
+using sm100::pdl_wait;
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
@@ -603,6 +607,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist, int hstride, DevErr* err) {
   __shared__ unsigned int hist[kBins];
+  pdl_launch_dependents();
+  pdl_wait();
   const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
   int b, t, n;
   const float* row;
@@ -624,6 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, 
 // histogram, write the keys above B, append bin B's keys to the candidates.
 __global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
   __shared__ unsigned int hist[kBins];
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ unsigned int warp_tot[kWarps];
   __shared__ unsigned int s_bin, s_above, s_total;
   const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
@@ -722,6 +730,9 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs 
 // passes over the row.
 __global__ void __launch_bounds__(kThreads, 2) topk_seg_final_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
   extern __shared__ uint8_t smem_raw[];
+  // the decode attention may start its prologue now on the idle SMs
+  pdl_launch_dependents();
+  pdl_wait();
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   int b, t, n;
   const float* row;
@@ -836,10 +847,16 @@ __global__ void topk_fill_kernel(TopkArgs a, DevErr* err) {
 }
 
 // Zero the first `words` words of each of `rows` rows of `stride` words.
+// Launched as a programmatic dependent of the indexer, it clears the
+// histograms while the scores are still being written, then waits for the
+// indexer so that its own completion implies the scores' (the histogram
+// kernel after it waits for this grid only).
 __global__ void topk_zero_kernel(unsigned int* p, int rows, int stride, int words) {
+  pdl_launch_dependents();
   const size_t n = (size_t)rows * words;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
     p[(i / words) * stride + i % words] = 0u;
+  pdl_wait();
 }
 
 }  // namespace
@@ -869,13 +886,22 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
     note_launches(1);
     return cudaGetLastError();
   }
+  // four launches, each a programmatic dependent of the one before (the
+  // first of the indexer's): each starts while its predecessor drains
   unsigned int* w = static_cast<unsigned int*>(ws);
-  topk_zero_kernel<<<64, 256, 0, c.stream>>>(w, rows, kWsRowWords, kWsKeys);
-  topk_seg_hist_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, kWsRowWords, c.err);
-  topk_seg_collect_kernel<<<rows * kSegBlocks, kThreads, 0, c.stream>>>(a, w, c.err);
   e = cudaFuncSetAttribute(topk_seg_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_seg_final_kernel<<<rows, kThreads, smem, c.stream>>>(a, w, c.err);
+  if ((e = launch_pdl(topk_zero_kernel, dim3(64), dim3(256), 0, c.stream, w, rows, (int)kWsRowWords,
+                      (int)kWsKeys)) != cudaSuccess)
+    return e;
+  if ((e = launch_pdl(topk_seg_hist_kernel, dim3(rows * kSegBlocks), dim3(kThreads), 0, c.stream, a, w,
+                      (int)kWsRowWords, c.err)) != cudaSuccess)
+    return e;
+  if ((e = launch_pdl(topk_seg_collect_kernel, dim3(rows * kSegBlocks), dim3(kThreads), 0, c.stream, a, w, c.err)) !=
+      cudaSuccess)
+    return e;
+  if ((e = launch_pdl(topk_seg_final_kernel, dim3(rows), dim3(kThreads), smem, c.stream, a, w, c.err)) != cudaSuccess)
+    return e;
   note_launches(4);
   return cudaGetLastError();
 }
