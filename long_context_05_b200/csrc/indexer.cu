@@ -634,9 +634,20 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   };
   p.kc = kKC;
   long long items = count_items(p.kc);
-  while (p.kc > 4 && items < 4LL * c.num_sms) {
-    p.kc /= 2;
-    items = count_items(p.kc);
+  if (items < 4LL * c.num_sms) {
+    // few items (decode: one query group per sequence): the key-run length
+    // that gives the busiest CTA the fewest key tiles, then the fewest items
+    // (each item reloads its queries and weights)
+    long long best = -1;
+    for (int kc = kKC; kc >= 4; --kc) {
+      const long long n = count_items(kc);
+      const long long load = (n + c.num_sms - 1) / c.num_sms * kc;
+      if (best < 0 || load < best) {
+        best = load;
+        p.kc = kc;
+        items = n;
+      }
+    }
   }
   const int grid = (int)(items < c.num_sms ? items : c.num_sms);
   if (grid <= 0) return cudaSuccess;
