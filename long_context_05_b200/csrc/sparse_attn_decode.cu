@@ -29,9 +29,9 @@
 //     copying three of the nine atoms of every row with 16-byte cp.async);
 //     warps 7-14 run the softmax (two per TMEM lane quarter, one per half,
 //     exchanging partial maxima and sums through shared memory) and drain O.
-// Q K^T of each 64-key half starts as soon as that half has landed; P V runs
-// in four 128-column quarters (N = 128, K = the 128 keys) so the read-out of
-// one quarter overlaps the MMAs of the next.  Each split writes its output
+// Q K^T runs once both 64-key halves have landed, as one N = 128 pass over
+// the split's keys; P V runs in four 128-column quarters (N = 128, K = the
+// 128 keys) so the read-out of one quarter overlaps the MMAs of the next.  Each split writes its output
 // normalised by its own row sum, as FP16 (|O| is bounded by the largest |V|,
 // far inside FP16's range, and FP16 keeps 11 significant bits), with its
 // log2-sum-exp in FP32; a combine kernel, launched as a programmatic
@@ -235,23 +235,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc(kFmtBF16, kFmtBF16, 0, 0, 128, kChunk);
+      constexpr uint32_t idesc_qk = make_idesc(kFmtBF16, kFmtBF16, 0, 0, 128, 2 * kChunk);
       constexpr uint32_t idesc_pv = make_idesc(kFmtBF16, kFmtBF16, 0, 1, 128, 128);
       const uint64_t kdesc0 = make_sdesc(smem_u32(sKV), 16, 1024, kSwizzle128);
       const uint64_t qdesc0 = make_sdesc(smem_u32(sQ), 16, 1024, kSwizzle128);
       bool ok = row_ok && mbar_wait(q_full, 0, p.wait_ns, ab) && mbar_wait(q_ready, 0, p.wait_ns, ab);
       if (!ok && row_ok) fail(1);
       int issued_qk = 0, issued_pv = 0;
-      for (int c = 0; c < 2 && ok; ++c) {
-        if (!mbar_wait(&kv_full[c], 0, p.wait_ns, ab)) { fail(2); ok = false; break; }
+      // Q K^T over all 128 keys of the split as one N = 128 pass (36 MMAs
+      // instead of two N = 64 passes of 36: an N = 64 MMA costs the issuing
+      // thread nearly as much as an N = 128 one); both halves land together
+      if (ok && (!mbar_wait(&kv_full[0], 0, p.wait_ns, ab) || !mbar_wait(&kv_full[1], 0, p.wait_ns, ab))) {
+        fail(2);
+        ok = false;
+      }
+      if (ok) {
         fence_proxy_async_smem();
         tc_fence_after();
-        const uint32_t dS = tmem + kSCol + c * kChunk;
+        const uint32_t dS = tmem + kSCol;
 #pragma unroll
         for (int ks = 0; ks < kKSteps; ++ks) {
           const int d = ks * 16;
-          const uint64_t bdesc =
-              kdesc0 + (uint64_t)(((d / 64) * kAtomBytes + (d % 64) * 2 + c * kChunk * 128) >> 4);
+          const uint64_t bdesc = kdesc0 + (uint64_t)(((d / 64) * kAtomBytes + (d % 64) * 2) >> 4);
           if (ks < kQTSteps) {
             mma_bf16_ts(dS, tmem + kQCol + ks * 8, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
           } else {
@@ -260,8 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16(dS, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
           }
         }
-        mma_commit(&s_full[c]);
-        ++issued_qk;
+        // one commit per softmax side (each waits for its half's logits)
+        mma_commit(&s_full[0]);
+        mma_commit(&s_full[1]);
+        issued_qk = 2;
       }
       if (ok && !mbar_wait(p_full, 0, p.wait_ns, ab)) { fail(3); ok = false; }
       for (int q = 0; q < 4 && ok; ++q) {
