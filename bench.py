@@ -16,7 +16,10 @@ Kernel timing: each step calls the C-ABI step entry points in the order
 dsa_forward uses with a full workspace, with CUDA events between launches on
 the launching stream, so every kernel's share of the step is measured live;
 `e2e` runs dsa_forward itself on host (pinned) buffers with the copies inside
-the timed region.  `alternatives.select_fused` times dsa_select over the same
+the timed region: for a long single-sequence prefill, one call per 4096-row
+query block (a chunked prefill, seqlens = the block's end) with the copies of
+the next block's queries and of the finished blocks' outputs overlapping the
+compute on two copy streams; otherwise one call between the copies.  `alternatives.select_fused` times dsa_select over the same
 query blocks on its own (the fused indexer + top-k that dsa_forward takes when
 its workspace has no room for the score tile); it is not part of the step.
 
@@ -542,6 +545,81 @@ def run_e2e(runner, steps, ws):
     return ms, h2d, d2h
 
 
+def run_e2e_pipelined(runner, steps, ws):
+    """dsa_forward on pinned host buffers, one call per query block of
+    q_block rows (a chunked prefill: seqlens = the block's end, the whole key
+    cache as S), with the host->device copies of the next block's queries and
+    the device->host copies of the finished blocks' outputs on two copy
+    streams overlapping the compute.  Every step still copies all inputs in
+    and out + lse back; the per-block calls run the same kernels over the
+    same keys as one call over all rows (the first block's rows that keep
+    every key go through the top-k's fill instead of the dense shortcut)."""
+    d, wl = runner.dsa, runner.wl
+    qb = wl.q_block
+    blocks = [(s0, min(qb, wl.T - s0)) for s0 in range(0, wl.T, qb)]
+    key_names = ("k_I", "k_scale", "kv")
+    q_names = ("q_I", "q_scale", "w", "q")
+    host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in runner.inp.items()}
+    for k, v in runner.inp.items():
+        host_in[k].copy_(v)
+    o = runner.outs
+    host_out = torch.empty(o.out.shape, dtype=torch.bfloat16, pin_memory=True)
+    host_lse = torch.empty(o.lse.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4
+    ends = [torch.tensor([s0 + c], dtype=torch.int32, device="cuda") for s0, c in blocks]
+    shapes = [d.make_shape(wl.with_(T=c, q_block=c), mode=d.DSA_PREFILL, seqlens=e)
+              for (s0, c), e in zip(blocks, ends)]
+    ws_blk = d.alloc_workspace(shapes[0])
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    def one():
+        main = torch.cuda.current_stream()
+        for st in (s_in, s_cmp, s_out):
+            st.wait_stream(main)
+        ev_in = []
+        with torch.cuda.stream(s_in):
+            for n in key_names:
+                runner.inp[n].copy_(host_in[n], non_blocking=True)
+            for s0, c in blocks:
+                for n in q_names:
+                    runner.inp[n][:, s0:s0 + c].copy_(host_in[n][:, s0:s0 + c], non_blocking=True)
+                ev_in.append(torch.cuda.Event())
+                ev_in[-1].record(s_in)
+        ev_done = []
+        with torch.cuda.stream(s_cmp):
+            for (s0, c), shape, ev in zip(blocks, shapes, ev_in):
+                s_cmp.wait_event(ev)
+                part = {n: runner.inp[n][:, s0:s0 + c] for n in q_names}
+                part.update({n: runner.inp[n] for n in key_names})
+                d.forward(shape, part, o.out[:, s0:s0 + c], o.lse[:, s0:s0 + c], o.idx[:, s0:s0 + c], ws_blk)
+                ev_done.append(torch.cuda.Event())
+                ev_done[-1].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            for (s0, c), ev in zip(blocks, ev_done):
+                s_out.wait_event(ev)
+                host_out[:, s0:s0 + c].copy_(o.out[:, s0:s0 + c], non_blocking=True)
+                host_lse[:, s0:s0 + c].copy_(o.lse[:, s0:s0 + c], non_blocking=True)
+        main.wait_stream(s_out)
+
+    one()
+    torch.cuda.synchronize()
+    st, det = d.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {det:#x}")
+    barrier(ws)
+    s0e = torch.cuda.Event(enable_timing=True)
+    s1e = torch.cuda.Event(enable_timing=True)
+    s0e.record()
+    for _ in range(steps):
+        one()
+    s1e.record()
+    s1e.synchronize()
+    ms = max_over_ranks(s0e.elapsed_time(s1e) / steps, ws)
+    del host_in
+    return ms, h2d, d2h, len(blocks)
+
+
 def gpu_arm(args):
     ws, rank, local = dist_setup(args.gpus)
     from long_context_05_b200 import dsa
@@ -606,9 +684,15 @@ def gpu_arm(args):
     if not args.no_e2e and avail is not None and avail < 2 * need * max(1, ws):
         e2e = {"skipped": f"host RAM available {avail / 2**30:.0f} GiB < 2 x {need / 2**30:.0f} GiB pinned per rank"}
     elif not args.no_e2e:
-        e_ms, h2d, d2h = run_e2e(runner, args.e2e_steps, ws)
+        if not wl.decode and wl.B == 1 and wl.T > wl.q_block:
+            # a long prefill: per-block calls with the copies overlapping
+            e_ms, h2d, d2h, nblk = run_e2e_pipelined(runner, args.e2e_steps, ws)
+            how = f"dsa_forward per {wl.q_block}-row query block ({nblk} calls), copies on two streams overlapping"
+        else:
+            e_ms, h2d, d2h = run_e2e(runner, args.e2e_steps, ws)
+            how = "one dsa_forward call between the copies"
         e2e = {"value": ws * wl.B * wl.T / (e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps, "how": how}
 
     rep = kernel_report(runner.wl, per_kernel, args.steps, peaks, peak_src, sustained=True)
     top = max(rep.items(), key=lambda kv: kv[1]["ms_per_step"])
