@@ -128,6 +128,10 @@ SMALL = [
              k=256, q_block=1, seed=10, needles=16),
     Workload("decode_k_covers_all", B=2, T=1, S=777, H_I=32, D_I=32, H=8, d_k=80, d_v=64,
              k=2048, q_block=1, seed=11),
+    # decode with fewer than 128 heads on the MLA row (the decode kernel's
+    # masked head rows) and a selection that ends inside its last split
+    Workload("decode_h64_ragged_k", B=2, T=1, S=3000, H_I=16, D_I=128, H=64, d_k=576, d_v=512,
+             k=1000, q_block=1, seed=12, needles=8),
 ]
 
 
