@@ -171,7 +171,9 @@ __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, 
 // score rows (no per-sequence lengths, stride 1, no thresholds, no repair
 // list); the general form adds lengths, paged caches, the key sample, the
 // candidate and the repair modes, whose checks the plain form must not pay.
-template <int DI, int HI, bool PLAIN>
+// CAND: candidate mode (thr set).  With PLAIN it keeps the contiguous
+// fast paths while appending candidates instead of storing scores.
+template <int DI, int HI, bool PLAIN, bool CAND>
 __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                       IdxParams p) {
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   constexpr int QPS = kNSub / HI;
   // the plain form sees constants: no sample stride, no candidates, no repair
   const int KS = PLAIN ? 1 : p.kstride;
-  const unsigned int* const THR = PLAIN ? nullptr : p.thr;
+  const unsigned int* const THR = CAND ? p.thr : nullptr;
   const int* const SLOT = PLAIN ? nullptr : p.row_slot;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -504,7 +506,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
               for (int i = 0; i < NP; ++i) a += part[g][q][i].x + part[g][q][i].y;
               const int t = it.t0 + j * QPS + q;
               const bool vis = t < it.tend && sp <= it.off + t;
-              if constexpr (PLAIN) {
+              if constexpr (PLAIN && !CAND) {
                 if (vis) {
                   // self-check: the score slot lies inside this launch's tile
                   const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
@@ -513,7 +515,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
                   else
                     report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_INDEXER | (1u << 8));
                 }
-              } else if (THR == nullptr) {
+              } else if constexpr (!CAND) {
                 if (vis) {
                   // self-check: the score slot lies inside this launch's tile
                   const long long ri = (long long)it.b * p.q_count + (t - p.q_begin);
@@ -651,9 +653,12 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   }
   const int grid = (int)(items < c.num_sms ? items : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  const bool plain =
-      ks == 1 && p.thr == nullptr && p.row_slot == nullptr && a.kv.page_size == 0 && a.kv.seqlens == nullptr;
-  auto kern = plain ? indexer_tc_kernel<DI, HI, true> : indexer_tc_kernel<DI, HI, false>;
+  // the contiguous fast paths (no lengths, no paging, stride 1, no repair
+  // list), with score rows or candidate lists as the output
+  const bool plain = ks == 1 && p.row_slot == nullptr && a.kv.page_size == 0 && a.kv.seqlens == nullptr;
+  const bool cand = p.thr != nullptr;
+  auto kern = cand ? (plain ? indexer_tc_kernel<DI, HI, true, true> : indexer_tc_kernel<DI, HI, false, true>)
+                   : (plain ? indexer_tc_kernel<DI, HI, true, false> : indexer_tc_kernel<DI, HI, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   kern<<<grid, EpiCfg<HI>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
