@@ -565,20 +565,34 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // The epilogue warps' candidate lists into per-row lists: one block per
-// warp list, one returning atomic per entry (latency hidden by the many
-// blocks in flight, away from the indexer's epilogue).
+// warp list.  The indexer appends 32 consecutive keys of one query at a time,
+// so neighbouring entries mostly share a row: the lanes of a warp holding the
+// same row reserve their slots with one returning atomic (the lowest such
+// lane adds the group's size), latency hidden by the many blocks in flight.
 __global__ void __launch_bounds__(256)
     topk_scatter_kernel(const int32_t* wl_row, const int32_t* wl_idx, const unsigned int* wl_key,
                         const unsigned int* wl_cnt, long long wl_cap, unsigned int* cnt, unsigned int* cand_key,
                         int32_t* cand_idx, int cap) {
   const long long base = (long long)blockIdx.x * wl_cap;
   const long long n = min((long long)wl_cnt[blockIdx.x], wl_cap);
-  for (long long i = threadIdx.x; i < n; i += 256) {
-    const int r = wl_row[base + i];
-    const unsigned int pos = atomicAdd(&cnt[r], 1u);
-    if (pos < (unsigned int)cap) {
-      cand_key[(size_t)r * cap + pos] = wl_key[base + i];
-      cand_idx[(size_t)r * cap + pos] = wl_idx[base + i];
+  const int lane = threadIdx.x & 31;
+  // every thread runs the same number of rounds (whole warps take part in
+  // the match); lanes past the end hold row -1 and take no slot
+  for (long long i0 = 0; i0 < n; i0 += 256) {
+    const long long i = i0 + threadIdx.x;
+    const bool valid = i < n;
+    const int r = valid ? wl_row[base + i] : -1;
+    const unsigned int same = __match_any_sync(0xffffffffu, r);
+    const int leader = __ffs(same) - 1;
+    unsigned int first = 0u;
+    if (valid && lane == leader) first = atomicAdd(&cnt[r], (unsigned int)__popc(same));
+    first = __shfl_sync(0xffffffffu, first, leader);
+    if (valid) {
+      const unsigned int pos = first + (unsigned int)__popc(same & ((1u << lane) - 1u));
+      if (pos < (unsigned int)cap) {
+        cand_key[(size_t)r * cap + pos] = wl_key[base + i];
+        cand_idx[(size_t)r * cap + pos] = wl_idx[base + i];
+      }
     }
   }
 }
