@@ -143,8 +143,8 @@ DSA_API size_t dsa_workspace_size(const dsa_shape* shape);
 
 /* Bytes of workspace for dsa_select, and the least a prefill dsa_forward
  * accepts, where the fused selection applies (prefill, contiguous caches,
- * S >= 32768, S a multiple of 16): its regions replace the score tile, about
- * a third of the tile's size (0.64 GiB instead of 2 GiB for a 4096-row block
+ * S >= 32768, S a multiple of 32): its regions replace the score tile, about
+ * a quarter of the tile's size (0.56 GiB instead of 2 GiB for a 4096-row block
  * of a 128K context).  Elsewhere equal to dsa_workspace_size.  0 if the shape
  * is invalid. */
 DSA_API size_t dsa_select_workspace_size(const dsa_shape* shape);
@@ -182,11 +182,11 @@ DSA_API dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
 /* Steps A and B together for queries [q_begin, q_begin + q_count): writes the
  * selection idx[b, t, 0..k) as dsa_topk does (ties to the lower index, -1
  * after the last).  ws: dsa_select_workspace_size(shape) bytes.
- * In prefill over long contexts (S >= 32768, S a multiple of 16, contiguous
+ * In prefill over long contexts (S >= 32768, S a multiple of 32, contiguous
  * caches) the query block's score matrix is never stored (the pages ask that
  * the selection be cache-aware and stay on the device: sider.ai blog on
  * DeepSeek Sparse Attention, "Uyarilar"): the
- * indexer scores every 16th key, a per-row radix select on that sample gives
+ * indexer scores every 32nd key, a per-row radix select on that sample gives
  * a threshold expected to admit about 2k keys, the indexer then scores every
  * key and keeps only (score, index) pairs at or above the row's threshold
  * (at most 8192 per row), and the top k are selected exactly among them.  A

@@ -127,7 +127,7 @@ float tau_of(const dsa_shape* s) {
 
 // Selection without a score tile: prefill over long contexts with a
 // contiguous key cache (the sample reads every kSampleStride-th cache row).
-constexpr int kSampleStride = 16;
+constexpr int kSampleStride = 32;
 constexpr int kRepairRows = 64;   // rows of one block that can fall back to a materialised score row
 constexpr int kTargetNum = 3, kTargetDen = 2;   // about 1.5 k candidates expected per row
 constexpr int kRowCap = 6144;     // candidates a row's list holds (<= the top-k's shared capacity)

@@ -114,7 +114,7 @@ def _adversarial(kind):
         inp["k_scale"][:] = inp["k_scale"][:, :1].clone()
     else:
         keep = torch.zeros(wl.S, dtype=torch.bool, device="cuda")
-        keep[::16] = True                                     # the rows the 16-stride sample reads
+        keep[::32] = True                                     # the rows the 32-stride sample reads
         inp["k_I"][:, ~keep] = 0                              # score exactly 0 elsewhere
     return wl, inp
 
