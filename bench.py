@@ -22,6 +22,11 @@ the next block's queries and of the finished blocks' outputs overlapping the
 compute on two copy streams; otherwise one call between the copies.  `alternatives.select_fused` times dsa_select over the same
 query blocks on its own (the fused indexer + top-k that dsa_forward takes when
 its workspace has no room for the score tile); it is not part of the step.
+`extras` (one GPU only; --no-extras skips it) times the path's other forms
+the same way: the decode over page pools against the contiguous one, the
+dense attention beside the sparse one on the 8K prefill plus a short prefill
+that dsa_forward runs wholly in the dense form, and one indexer training step
+(scores, KL target, KL loss, backward) in its sparse and warm-up stages.
 
 Inputs are synthetic (long_context_05_b200.inputs), larger than L2 for the
 prefill; L2 is flushed between timed steps anyway (a 256 MiB write outside
@@ -46,7 +51,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from long_context_05_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+from long_context_05_b200.inputs import WORKLOADS, make_inputs, to_paged  # noqa: E402
 from long_context_05_b200.parallel import barrier as _barrier, max_over_ranks as _max_over_ranks  # noqa: E402
 from long_context_05_b200.parallel import rank_seed  # noqa: E402
 
@@ -83,6 +88,9 @@ def measured_traffic(workload: str, kernel: str):
     return t["bytes"]
 FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# FP32 FMA issue on CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
+# (clocks.max.sm); the peak of kernels that run plain FP32 arithmetic
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
 
 
 # ------------------------------------------------------------------ helpers
@@ -213,13 +221,18 @@ def scored_pairs(wl):
 class DsaRunner:
     """Runs one workload through the C ABI, step by step, with events."""
 
-    def __init__(self, wl, seed_offset=0):
+    def __init__(self, wl, seed_offset=0, page_size=0):
         from long_context_05_b200 import dsa
         self.dsa = dsa
         self.wl = wl = wl.with_(seed=rank_seed(wl.seed, seed_offset))
         self.inp = make_inputs(wl, "cuda")
         self.inp.pop("needle_pos", None)
-        self.shape = dsa.make_shape(wl)
+        if page_size:
+            # key-side caches in page pools, pages in a random order
+            self.inp, self.table, num_pages = to_paged(self.inp, wl, page_size, wl.seed)
+            self.shape = dsa.make_shape(wl, block_table=self.table, page_size=page_size, num_pages=num_pages)
+        else:
+            self.shape = dsa.make_shape(wl)
         self.ws = dsa.alloc_workspace(self.shape)
         self.outs = dsa.alloc_outputs(wl)
         self.ld = (wl.S + 63) // 64 * 64
@@ -620,6 +633,186 @@ def run_e2e_pipelined(runner, steps, ws):
     return ms, h2d, d2h, len(blocks)
 
 
+# ------------------------------------------------------------------ other forms of the path
+
+class CallRunner:
+    """A list of named launch groups run as one step (the time_steps protocol:
+    .dsa, .step(ev))."""
+
+    def __init__(self, dsa, groups):
+        self.dsa = dsa
+        self.groups = groups
+
+    def step(self, ev=None):
+        for name, fn in self.groups:
+            if ev is None:
+                fn()
+                continue
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ev.append((name, a, b))
+
+
+def part_report(ms, amount, unit, bound, peak, note):
+    achieved = amount / (ms / 1e3)
+    return {"ms_per_step": ms, "bound": bound, "achieved": achieved, "unit": unit, "peak": peak,
+            "frac": achieved / peak, "peak_note": note,
+            "work_per_step": amount * (1e12 if unit == "TFLOP/s" else 1e9)}
+
+
+def timed_groups(runner, steps, warmup, ws):
+    total, per, launches = time_steps(runner, steps, warmup, ws)
+    return (max_over_ranks(total / steps, ws), {n: sum(v) / steps for n, v in per.items()}, launches // steps)
+
+
+def extra_paged_decode(wl, steps, warmup, ws, peaks, peak_src, contiguous_ms, page_size=64):
+    """Decode over page pools (random page order) against the contiguous
+    caches: the same work, so the ratio is the paging cost."""
+    run = DsaRunner(wl, page_size=page_size)
+    got = capture_step_graphs(run, warmup)
+    if got is not None:
+        total, kern = time_graphs(got[0], steps, warmup, ws)
+        launches, timing = got[1], "cuda_graph_replay"
+        got[0].clear()
+        torch.cuda.synchronize()
+    else:
+        total, kern, launches = time_steps(run, steps, warmup, ws)
+        launches //= steps
+        timing = "eager"
+    ms = max_over_ranks(total / steps, ws)
+    rep = kernel_report(run.wl, kern, steps, peaks, peak_src, sustained=False)
+    for r in rep.values():
+        r.pop("share", None)
+    del run
+    return {"workload": f"{wl.name} paged", "page_size": page_size, "value": ws * wl.B * wl.T / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_step": ms, "timing": timing, "gpu_launches": launches,
+            "vs_contiguous": ms / contiguous_ms if contiguous_ms else None, "kernels": rep}
+
+
+def extra_dense(wl, steps, warmup, ws, peaks, peak_src):
+    """dsa_dense_attn (every visible key) beside the sparse attention over the
+    selected keys, on the same queries and cache; and dsa_forward on a prefill
+    short enough that every row keeps all its visible keys (the whole call is
+    the dense form)."""
+    from long_context_05_b200 import dsa
+    bf16 = peaks["bf16_tflops_sustained"]
+    run = DsaRunner(wl)
+    run.step()
+    i, o = run.inp, run.outs
+    dout = torch.empty_like(o.out)
+    dlse = torch.empty_like(o.lse)
+    cr = CallRunner(dsa, [("sparse_attn", lambda: dsa.sparse_attn(run.shape, i["q"], i["kv"], o.idx, o.out, o.lse,
+                                                                  run.ws)),
+                          ("dense_attn", lambda: dsa.dense_attn(run.shape, i["q"], i["kv"], dout, dlse, run.ws))])
+    ms, per, launches = timed_groups(cr, steps, warmup, ws)
+    ip, ap = causal_pairs(wl)
+    fl = 2.0 * wl.H * (wl.d_k + wl.d_v)
+    note = f"bf16 sustained ({peak_src})"
+    res = {"workload": wl.name, "gpu_launches": launches,
+           "sparse_attn": part_report(per["sparse_attn"], fl * ap / 1e12, "TFLOP/s", "tensor", bf16, note),
+           "dense_attn": part_report(per["dense_attn"], fl * ip / 1e12, "TFLOP/s", "tensor", bf16, note)}
+    res["dense_vs_sparse_ms"] = per["dense_attn"] / per["sparse_attn"]
+    del run, cr
+    # a short prefill: k covers every row, so dsa_forward runs the dense form
+    swl = wl.with_(name=f"prefill_{wl.k // 1024}k_b4", B=4, T=wl.k, S=wl.k, q_block=wl.k)
+    srun = DsaRunner(swl)
+    cr = CallRunner(dsa, [("forward", srun.forward)])
+    ms, per, launches = timed_groups(cr, steps, warmup, ws)
+    ip, _ = causal_pairs(swl)
+    res["short_prefill"] = {"workload": swl.name, "config": {"batch": swl.B, "seq_len": swl.T, "k": swl.k},
+                            "value": ws * swl.B * swl.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+                            "gpu_launches": launches,
+                            "roofline": part_report(ms, fl * ip / 1e12, "TFLOP/s", "tensor", bf16, note)}
+    del srun, cr
+    return res
+
+
+def extra_train(wl, steps, warmup, ws, peaks, peak_src):
+    """One indexer training step over all query rows, per query block: the
+    indexer's scores, the KL target from the main attention, the KL loss and
+    dL/dI, and the backward to q_I, w and k_I.  Sparse stage (the selected
+    set, lse from the sparse attention) and warm-up (every visible key, lse
+    from the dense attention)."""
+    from long_context_05_b200 import dsa
+    run = DsaRunner(wl)
+    run.step()
+    i, o = run.inp, run.outs
+    qb = min(wl.q_block, wl.T)
+    rows = wl.B * qb
+    ld = run.ld
+    target = torch.zeros(rows, ld, device="cuda")
+    grad = torch.zeros(rows, ld, device="cuda")
+    loss = torch.zeros(rows, device="cuda")
+    dq = torch.zeros(wl.B, wl.T, wl.H_I, wl.D_I, device="cuda")
+    dw = torch.zeros(wl.B, wl.T, wl.H_I, device="cuda")
+    dk = torch.zeros(wl.B, wl.S, wl.D_I, device="cuda")
+    dout = torch.empty_like(o.out)
+    dlse = torch.empty_like(o.lse)
+    dsa.dense_attn(run.shape, i["q"], i["kv"], dout, dlse, run.ws)
+    sh = run.shape
+
+    def groups(idx, lse):
+        g = [("dk_zero", dk.zero_)]
+        for q0 in range(0, wl.T, qb):
+            cnt = min(qb, wl.T - q0)
+            g += [("indexer", lambda q0=q0, cnt=cnt: dsa.indexer_scores(
+                      sh, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], q0, cnt, run.scores)),
+                  ("kl_target", lambda q0=q0, cnt=cnt: dsa.kl_target(sh, i["q"], i["kv"], lse, q0, cnt, target, idx)),
+                  ("indexer_kl", lambda q0=q0, cnt=cnt: dsa.indexer_kl(sh, run.scores, target, q0, cnt, grad, loss,
+                                                                       idx)),
+                  ("indexer_backward", lambda q0=q0, cnt=cnt: dsa.indexer_backward(
+                      sh, i["q_I"], i["q_scale"], i["w"], i["k_I"], i["k_scale"], grad, q0, cnt, dq, dw, dk, idx))]
+        return g
+
+    ip, ap = causal_pairs(wl)
+    bf16 = peaks["bf16_tflops_sustained"]
+    res = {}
+    for stage, idx, lse, pairs in (("sparse", o.idx, o.lse, ap), ("warmup_dense", None, dlse, ip)):
+        cr = CallRunner(dsa, groups(idx, lse))
+        ms, per, launches = timed_groups(cr, steps, warmup, ws)
+        # per row: the set's scores and targets read, grad written over the visible keys
+        kl_bytes = (8.0 * pairs + 4.0 * ip) if idx is not None else 12.0 * ip
+        parts = {
+            "indexer": part_report(per["indexer"], 2.0 * wl.H_I * wl.D_I * ip / 1e12, "TFLOP/s", "tensor",
+                                   bf16 * FP8_PER_BF16, f"fp8 = sustained bf16 x {FP8_PER_BF16:g} ({peak_src})"),
+            "kl_target": part_report(per["kl_target"], 2.0 * wl.H * wl.d_k * pairs / 1e12, "TFLOP/s", "tensor",
+                                     bf16, f"bf16 sustained ({peak_src}); Q K^T of the set"),
+            "indexer_kl": part_report(per["indexer_kl"], kl_bytes / 1e9, "GB/s", "hbm", peaks["hbm_gbs"],
+                                      f"hbm ({peak_src}); scores + target of the set read, grad row written"),
+            "indexer_backward": part_report(per["indexer_backward"], 6.0 * wl.H_I * wl.D_I * pairs / 1e12,
+                                            "TFLOP/s", "alu", FP32_ALU_TFLOPS,
+                                            "fp32 FMA, 148 SMs x 128 lanes at 1965 MHz; D, dq and dk per pair"),
+        }
+        res[stage] = {"ms_per_step": ms, "rows_per_s": ws * wl.B * wl.T / (ms / 1e3), "gpu_launches": launches,
+                      "kernels": parts}
+    st, det = dsa.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {det:#x}")
+    del run
+    res["workload"] = wl.name
+    return res
+
+
+def run_extras(args, ws, peaks, peak_src, contiguous_decode_ms):
+    """The forms of the path beside the headline step, each timed on its own
+    with the same warm-up, flushes and events: paged decode, the dense form,
+    and the indexer's training step."""
+    steps, warmup = max(2, args.steps), args.warmup
+    out = {}
+    if args.decode_workload != "none":
+        out["paged_decode"] = extra_paged_decode(WORKLOADS[args.decode_workload], steps, warmup, ws, peaks, peak_src,
+                                                 contiguous_decode_ms)
+        torch.cuda.empty_cache()
+    out["dense"] = extra_dense(WORKLOADS["prefill_8k"], steps, warmup, ws, peaks, peak_src)
+    torch.cuda.empty_cache()
+    out["train"] = extra_train(WORKLOADS["prefill_8k"], steps, warmup, ws, peaks, peak_src)
+    torch.cuda.empty_cache()
+    return out
+
+
 def gpu_arm(args):
     ws, rank, local = dist_setup(args.gpus)
     from long_context_05_b200 import dsa
@@ -706,6 +899,15 @@ def gpu_arm(args):
         f["workspace_bytes"] = int(runner.ws_fused.numel())
         f["score_tile_workspace_bytes"] = int(runner.ws.numel())
         alternatives = {"select_fused": f}
+    # the other forms of the path, on one GPU only (each rank decides alike)
+    extras = None
+    if ws == 1 and not args.no_extras:
+        del runner
+        torch.cuda.empty_cache()
+        xclk = ClockSampler(local)
+        xclk.start()
+        extras = run_extras(args, ws, peaks, peak_src, dec["ms_per_step"] if dec else None)
+        extras["clocks"] = xclk.stop()
     tokens = ws * wl.B * wl.T
     line = {
         "metric": METRIC,
@@ -731,6 +933,7 @@ def gpu_arm(args):
         "kernels": rep,
         "alternatives": alternatives,
         "decode": dec,
+        "extras": extras,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clk,
@@ -783,6 +986,7 @@ def main():
     ap.add_argument("--decode-workload", default=DECODE, choices=sorted(WORKLOADS) + ["none"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()

@@ -249,3 +249,35 @@ def make_inputs(wl: Workload, device="cpu") -> dict:
             out["needle_pos"][b] = npos
     return out
 
+
+
+def to_paged(inp: dict, wl: Workload, page_size: int, seed: int):
+    """Scatter the key-side arrays of ``inp`` (k_I, k_scale, kv and v when
+    present) into page pools, pages in a random order.
+
+    Sequence b's page p (tokens p * page_size .. + page_size - 1) goes to pool
+    page table[b, p]; the pool has two spare pages that no sequence maps, and
+    the table one extra column of -1 (an unmapped page past each sequence's
+    last).  Returns (inputs with the pools in place of the key-side arrays,
+    int32 table [B, ppseq + 1] on the inputs' device, number of pool pages).
+    """
+    import numpy as np
+
+    ppseq = (wl.S + page_size - 1) // page_size
+    num_pages = wl.B * ppseq + 2
+    perm = np.random.default_rng(seed).permutation(num_pages)[: wl.B * ppseq].reshape(wl.B, ppseq)
+    table = np.full((wl.B, ppseq + 1), -1, np.int32)
+    table[:, :ppseq] = perm
+    dev = inp["kv"].device
+    # pool row of every (sequence, token): page base + offset in the page
+    rows = (torch.from_numpy(perm).to(dev, torch.int64).unsqueeze(-1) * page_size
+            + torch.arange(page_size, device=dev)).reshape(wl.B, -1)[:, : wl.S].reshape(-1)
+    out = dict(inp)
+    for name in ("k_I", "k_scale", "kv", "v"):
+        if name not in inp:
+            continue
+        x = inp[name]
+        pool = torch.zeros((num_pages * page_size,) + tuple(x.shape[2:]), dtype=x.dtype, device=dev)
+        pool[rows] = x.reshape((wl.B * wl.S,) + tuple(x.shape[2:]))
+        out[name] = pool
+    return out, torch.from_numpy(table).to(dev), num_pages

@@ -18,7 +18,7 @@ import pytest
 import torch
 
 from long_context_05_b200 import dsa
-from long_context_05_b200.inputs import Workload, make_inputs
+from long_context_05_b200.inputs import Workload, make_inputs, to_paged
 from oracle import dsa_oracle as O
 from tests import parity as P
 
@@ -154,27 +154,9 @@ def test_separate_values(wl):
 # ----------------------------------------------------------------- paged caches
 
 def _paged(inp, wl, page_size, seed):
-    """Scatter the key-side arrays of `inp` into page pools in a random page
-    order, with two spare pages and -1 past each sequence's pages."""
-    ppseq = (wl.S + page_size - 1) // page_size
-    num_pages = wl.B * ppseq + 2
-    rng = np.random.default_rng(seed)
-    perm = rng.permutation(num_pages)[: wl.B * ppseq].reshape(wl.B, ppseq)
-    table = np.full((wl.B, ppseq + 1), -1, np.int32)       # one unmapped page past the end
-    table[:, :ppseq] = perm
-    out = dict(inp)
-    for name in ("k_I", "k_scale", "kv", "v"):
-        if name not in inp:
-            continue
-        x = inp[name]
-        pool = torch.zeros((num_pages * page_size,) + tuple(x.shape[2:]), dtype=x.dtype, device="cuda")
-        for b in range(wl.B):
-            for p in range(ppseq):
-                s0, s1 = p * page_size, min(wl.S, (p + 1) * page_size)
-                r0 = int(perm[b, p]) * page_size
-                pool[r0: r0 + (s1 - s0)] = x[b, s0:s1]
-        out[name] = pool
-    return out, torch.from_numpy(table).cuda(), num_pages
+    """Key-side arrays in page pools, a random page order, spare pages and -1
+    past each sequence's pages."""
+    return to_paged(inp, wl, page_size, seed)
 
 
 PAGED = [
