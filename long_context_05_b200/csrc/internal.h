@@ -200,6 +200,13 @@ int indexer_epilogue_warps(int H_I);
 cudaError_t launch_topk_repair(const LaunchCtx& c, const TopkArgs& a, const float* tile, long long ld,
                                const int* fail_rows, const unsigned int* nfail, int max_fail);
 
+// the indexer's backward on tensor cores (indexer_bwd.cu): D_I 128, H_I <= 64
+bool indexer_bwd_tc_supported(int H_I, int D_I);
+cudaError_t launch_indexer_bwd_tc(const LaunchCtx& c, const KvMap& map, const uint8_t* q_I, const float* q_scale,
+                                  const float* w, const uint8_t* k_I, const float* k_scale, const float* grad,
+                                  long long ld, const int32_t* idx, int B, int T, int k, int H_I, int q_begin,
+                                  int q_count, float* dq, float* dw, float* dk);
+
 cudaError_t launch_wait_timeout_probe(const LaunchCtx& c);
 
 // shape validation and launch context of the public entry points (dsa_api.cu)

@@ -576,6 +576,14 @@ extern "C" dsa_status dsa_indexer_backward(const dsa_shape* s, const uint8_t* q_
   if ((st = api_make_ctx(stream, &c)) != DSA_OK) return st;
   if (q_count == 0) return DSA_OK;
   const KvMap map = api_kv_map(s);
+  // tensor-core form where it applies (16-byte aligned rows, cache rows that
+  // fit an int); the CUDA-core form otherwise
+  if (indexer_bwd_tc_supported(s->H_I, s->D_I) && aligned16(q_I) && aligned16(k_I) && aligned16(dq) &&
+      aligned16(dk) && map.pool_rows(s->B) < (1ll << 31)) {
+    const cudaError_t e = launch_indexer_bwd_tc(c, map, q_I, q_scale, w, k_I, k_scale, grad, ld, idx, s->B, s->T,
+                                                s->k, s->H_I, q_begin, q_count, dq, dw, dk);
+    return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  }
   cudaError_t e = cudaErrorInvalidValue;
 #define DSA_BWD(HI_, DI_)                                                                                          \
   if (s->H_I == HI_ && s->D_I == DI_)                                                                              \

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from long_context_05_b200 import dsa
-from long_context_05_b200.inputs import Workload, make_inputs
+from long_context_05_b200.inputs import Workload, make_inputs, to_paged
 from oracle import dsa_oracle as O
 from tests import parity as P
 
@@ -94,3 +94,84 @@ def test_indexer_training_step(sparse):
         _close(dwg[t], dw_r, 1e-3, f"dw t={t}")
         dk_ref[: pos + 1] += dk_r
     _close(dkg, dk_ref, 1e-3, "dk")
+
+
+# ----------------------------------------------------------------- backward alone, several shapes
+
+BWD_CASES = [
+    # name, B, T, S, H_I, k (None: every visible key), page size, ragged lengths
+    ("dense_b2_ragged_8tiles", 2, 24, 900, 64, None, 0, True),
+    ("sparse_k300_h32_paged64", 2, 16, 1100, 32, 300, 64, False),
+    ("dense_h16_one_query_block", 1, 8, 700, 16, None, 0, False),
+    ("sparse_k2048_h64_16tiles", 1, 4, 2600, 64, 2048, 0, False),
+]
+
+
+@pytest.mark.parametrize("name,B,T,S,H_I,k,page,ragged", BWD_CASES, ids=[c[0] for c in BWD_CASES])
+def test_indexer_backward_shapes(name, B, T, S, H_I, k, page, ragged):
+    """dsa_indexer_backward fed a random dL/dI, against the oracle's chain
+    rule.  Integer FP8 bytes with power-of-two scales keep every dot product
+    exact on both sides, so the ReLU mask is the same decision; the
+    tolerance, 2e-5 of the largest entry, is FP32 accumulation over a few
+    thousand terms (a gradient carried in plain BF16 would miss it by far)."""
+    wl = Workload(name, B=B, T=T, S=S, H_I=H_I, D_I=128, H=8, d_k=80, d_v=64, k=k or 64, q_block=T, seed=90,
+                  int_mode=True)
+    inp = make_inputs(wl, "cuda")
+    inp.pop("needle_pos", None)
+    gen = torch.Generator(device="cuda").manual_seed(91)
+    inp["q_scale"] = torch.exp2(torch.randint(-3, 4, inp["q_scale"].shape, device="cuda", generator=gen).float())
+    inp["k_scale"] = torch.exp2(torch.randint(-3, 4, inp["k_scale"].shape, device="cuda", generator=gen).float())
+    lengths = [S - 37 * b if ragged else S for b in range(B)]
+    sl = torch.tensor(lengths, dtype=torch.int32, device="cuda") if ragged else None
+    ld = (S + 63) // 64 * 64
+    rows = B * T
+    grad = torch.randn(rows, ld, device="cuda", generator=gen)
+    idx = None
+    rng = np.random.default_rng(92)
+    if k is not None:
+        sel = np.full((B, T, k), -1, np.int32)
+        for b in range(B):
+            for t in range(T):
+                n = lengths[b] - T + t + 1
+                keys = rng.choice(n, size=min(k, n), replace=False)
+                slots = rng.permutation(k)[: keys.size]         # valid keys anywhere in the row
+                sel[b, t, slots] = keys
+        idx = torch.from_numpy(sel).cuda()
+    key_inp = inp
+    if page:
+        key_inp, table, num_pages = to_paged(inp, wl, page, 93)
+        shape = dsa.make_shape(wl, seqlens=sl, block_table=table, page_size=page, num_pages=num_pages)
+        dk = torch.zeros(num_pages * page, wl.D_I, device="cuda")
+    else:
+        shape = dsa.make_shape(wl, seqlens=sl)
+        dk = torch.zeros(B, S, wl.D_I, device="cuda")
+    dq = torch.zeros(B, T, H_I, wl.D_I, device="cuda")
+    dw = torch.zeros(B, T, H_I, device="cuda")
+    dsa.indexer_backward(shape, inp["q_I"], inp["q_scale"], inp["w"], key_inp["k_I"], key_inp["k_scale"], grad, 0, T,
+                         dq, dw, dk, idx)
+    st, det = dsa.device_error()
+    assert st == 0, (st, hex(det))
+    g_np = grad.cpu().double().numpy()
+    dq_np, dw_np, dk_np = dq.cpu().numpy(), dw.cpu().numpy(), dk.cpu().numpy()
+    for b in range(B):
+        d = O.from_inputs({k_: v.cpu() for k_, v in inp.items()}, b)
+        dk_ref = np.zeros((S, wl.D_I))
+        for t in range(T):
+            pos = lengths[b] - T + t
+            g = g_np[b * T + t, : pos + 1].copy()
+            if idx is not None:
+                keep = np.zeros(pos + 1, bool)
+                s_ = sel[b, t]
+                keep[s_[s_ >= 0]] = True
+                g[~keep] = 0.0
+            dq_r, dw_r, dk_r = O.indexer_grads_row(d["qd"][t], d["w"][t], d["kd"], pos, g)
+            _close(dq_np[b, t], dq_r, 2e-5, f"dq b={b} t={t}")
+            _close(dw_np[b, t], dw_r, 2e-5, f"dw b={b} t={t}")
+            dk_ref[: pos + 1] += dk_r
+        if page:
+            tb = table.cpu().numpy()
+            s_all = np.arange(S)
+            got = dk_np[tb[b, s_all // page] * page + s_all % page]
+        else:
+            got = dk_np[b]
+        _close(got, dk_ref, 2e-5, f"dk b={b}")
