@@ -329,6 +329,12 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Arrive on *bar once every cp.async this thread issued so far has landed
+// (counts as one of the barrier's expected arrivals).  The consumer orders
+// the copied bytes before its tensor-core reads with fence_proxy_async_smem.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // ------------------------------------------------------------------ launch order
 

@@ -12,12 +12,14 @@
 //   dsa_kl_target:         p[t, s] = (1/H) sum_h exp(tau q_h . kv_s - lse_h)
 //                          with lse from the main attention (dense: every
 //                          visible key; sparse: the selected set, where lse
-//                          is the sparse attention's), on tcgen05: Q K^T of a
-//                          128-key split as in the decode kernel, then the
-//                          head sum in the epilogue;
+//                          is the sparse attention's), on tcgen05: one CTA
+//                          per query with Q resident in TMEM, Q K^T per
+//                          64-key chunk, the head sum in the epilogue;
 //   dsa_indexer_kl:        per row, loss and dL/dI = softmax(I) - p;
 //   dsa_indexer_backward:  dL/dw, dL/dq_I, dL/dk_I through the ReLU, on the
-//                          dequantised operands (FP32, CUDA cores).
+//                          dequantised operands: on tcgen05 for D_I = 128
+//                          (indexer_bwd.cu), FP32 on the CUDA cores here
+//                          otherwise.
 #include <cuda_fp8.h>
 #include <math.h>
 
@@ -32,23 +34,35 @@ using namespace sm100;
 
 // ------------------------------------------------------------------ KL target
 
+// One CTA per query row.  All of the row's Q (128 heads x 576 dims, BF16)
+// sits in TMEM for the whole row, so every MMA reads A from TMEM; it gets
+// there through the first two ring slots (each thread copies its own head
+// row in, swizzled so the read-back is free of bank conflicts) while the
+// first chunk of keys lands in the third.  The keys stream through the ring
+// of three 64-key slots (128B-swizzled K-major atoms laid out
+// [slot][atom][row]); chunk j uses slot (j + 2) mod 3.  Per 64-key chunk: S = Q K^T
+// (36 MMAs of 128 x 64 x 16) into one of two TMEM buffers, then the head sum
+// of exp(tau S - lse_h) on eight warps: each warp reduces its 32 heads for 32
+// keys with one transpose-reduce over the lanes (31 shuffles), the four lane
+// quarters meet in shared memory, and one warp per key half writes the row's
+// target entries.
 constexpr int DK = 576;
-constexpr int kKeys = 128, kChunk = 64, kNAtom = DK / 64, kAtomBytes = kKeys * 128;
-constexpr int kQT = 256, kQSAtoms = (DK - kQT) / 64, kQAtomBytes = 128 * 128;
-constexpr int kKSteps = DK / 16, kQTSteps = kQT / 16;
-constexpr uint32_t kTmemCols = 256, kSCol = 0, kQCol = 128;
+constexpr int kChunk = 64, kSlots = 3, kNAtom = DK / 64;
+constexpr int kAtomBytes = kChunk * 128, kSlotBytes = kNAtom * kAtomBytes;
+constexpr int kKSteps = DK / 16;
+constexpr uint32_t kTmemCols = 512, kQCol = 0, kSCol = 384;      // Q [0, 288), S x2 [384, 512)
 constexpr int kFirstGather = 1, kGatherWarps = 6, kFirstEpi = 7, kEpiWarps = 8;
 constexpr int kThreads = 32 * (kFirstEpi + kEpiWarps);
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + kQSAtoms * kQAtomBytes;
-constexpr int OFF_MASK = OFF_KV + kNAtom * kAtomBytes;
-constexpr int OFF_KEY = OFF_MASK + 16;                 // key of each slot (int32 [128])
-constexpr int OFF_SUM = OFF_KEY + kKeys * 4;           // head sums (float [128])
-constexpr int OFF_BAR = OFF_SUM + kKeys * 4;
-constexpr int kNumBars = 2 + 2 + 2 + 1;                // q_full, q_ready, kv_full[2], s_full[2], mma_done
+constexpr int kGatherThreads = 32 * kGatherWarps;
+constexpr int OFF_KV = 0;
+constexpr int OFF_SUM = OFF_KV + kSlots * kSlotBytes;     // head sums, two chunk buffers (float)
+constexpr int OFF_BAR = OFF_SUM + 2 * kChunk * 4;
+constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 1;       // q_ready, kv_full[3], kv_empty[3], s_full[2], s_empty[2], mma_done
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kSmem = OFF_MISC + 16;
 static_assert(kSmem <= 232448, "shared memory per CTA");
+static_assert(kGatherThreads == 3 * kChunk, "three gather threads per key row");
+static_assert(128 * DK * 2 <= 2 * kSlotBytes, "Q fits the first two slots");
 
 struct TargetParams {
   KvMap map;
@@ -59,56 +73,71 @@ struct TargetParams {
   float* target;
   long long ld;
   int T, H, k, q_begin, q_count, B;
-  int nsplit;
   float scale_log2;
+  bool tma_keys;          // every visible key, contiguous cache: chunks by TMA tiles
   long long wait_ns;
   DevErr* err;
 };
 
+// v[i] over the warp's lanes, summed: lane l returns sum over lanes of v[l]
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    kl_target_kernel(const __grid_constant__ CUtensorMap tm_q, TargetParams p) {
-  extern __shared__ uint8_t smem[];
+    kl_target_kernel(const __grid_constant__ CUtensorMap tm_kv, TargetParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (0xDu << 8));
     return;
   }
-  uint8_t* sQ = smem + OFF_Q;
   uint8_t* sKV = smem + OFF_KV;
-  uint64_t* sMask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
-  int* sKey = reinterpret_cast<int*>(smem + OFF_KEY);
   float* sSum = reinterpret_cast<float*>(smem + OFF_SUM);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* q_ready = bars + 1;
-  uint64_t* kv_full = bars + 2;
-  uint64_t* s_full = bars + 4;
-  uint64_t* mma_done = bars + 6;
+  uint64_t* q_ready = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + kSlots;
+  uint64_t* s_full = kv_empty + kSlots;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* mma_done = s_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int lr = blockIdx.x / p.nsplit;            // row of the launch: b * q_count + i
-  const int split = blockIdx.x - lr * p.nsplit;
+  const int lr = blockIdx.x;                       // row of the launch: b * q_count + i
   const int b = lr / p.q_count, t = p.q_begin + (lr - (lr / p.q_count) * p.q_count);
   const int row = b * p.T + t;                     // query row of the problem
   const int Lb = p.map.len(b, p.err, ERR_SITE_ATTN);
-  const int pos = Lb - p.T + t;
+  const int n = Lb - p.T + t + 1;                  // visible keys
   const bool dense = p.idx == nullptr;
-  const int slot0 = split * kKeys;
-  const int slot1 = min(dense ? pos + 1 : p.k, slot0 + kKeys);
+  const int m = dense ? n : p.k;                   // key slots of the row
+  const int nch = (m + kChunk - 1) / kChunk;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
     mbar_init(q_ready, kEpiWarps);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&kv_full[i], p.tma_keys ? 1 : kGatherThreads);
+      mbar_init(&kv_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 32 * (kGatherWarps / 2));
       mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kEpiWarps);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < kKeys; i += kThreads) sSum[i] = 0.f;
+  for (int i = threadIdx.x; i < 2 * kChunk; i += kThreads) sSum[i] = 0.f;
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -129,111 +158,128 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp >= kFirstGather && warp < kFirstEpi) {
-    // ------------------------------------------------------------ gather (as in the decode kernel)
-    const int g = warp - kFirstGather;
-    const int half = g / 3, sub = g - 3 * (g / 3);
-    bool q_issued = false;
-    if (g == 0 && lane == 0) {
-      prefetch_tmap(&tm_q);
-      mbar_arrive_expect_tx(q_full, kQSAtoms * kQAtomBytes);
-      for (int a = 0; a < kQSAtoms; ++a) tma_load_2d(sQ + a * kQAtomBytes, &tm_q, q_full, kQT + a * 64, row * p.H);
-      q_issued = true;
-    }
-    int iv2[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int slot = slot0 + half * kChunk + lane + 32 * u;
-      iv2[u] = slot < slot1 ? (dense ? slot : p.idx[(size_t)row * p.k + slot]) : -1;
-    }
-    const int c16 = lane & 7, rg = lane >> 3;
-    uint64_t mask = 0;
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll 2
-      for (int mm = 0; mm < 8; ++mm) {
-        const int m = 8 * u + mm;
-        const int r = rg + 4 * m;
-        int v = __shfl_sync(0xffffffffu, iv2[u], rg + 4 * mm);
-        if (v >= Lb) {
-          if (c16 == 0 && sub == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
-          v = -1;
+    const int gt = threadIdx.x - 32 * kFirstGather;
+    if (p.tma_keys) {
+      // ---------------------------------------------------------- keys 0.. of a contiguous cache: one
+      // thread loads each chunk as nine 64 x 64 tiles (rows past the cache read as zero)
+      if (gt == 0) {
+        prefetch_tmap(&tm_kv);
+        const int row0 = (int)p.map.row_contig(b, 0);
+        int issued = 0;
+        for (int j = 0; j < nch; ++j) {
+          const int sl = (j + 2) % kSlots;
+          if (j >= kSlots ? !mbar_wait(&kv_empty[sl], ((j / kSlots) - 1) & 1, p.wait_ns, ab)
+                          : (j >= 1 && !mbar_wait(q_ready, 0, p.wait_ns, ab))) {
+            fail(1);
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[sl], kSlotBytes);
+          for (int a = 0; a < kNAtom; ++a)
+            tma_load_2d(sKV + sl * kSlotBytes + a * kAtomBytes, &tm_kv, &kv_full[sl], a * 64, row0 + j * kChunk);
+          issued = j + 1;
         }
-        const long long cr = v >= 0 ? p.map.row(b, v) : -1;
-        if (v >= 0 && cr < 0) {
-          if (c16 == 0 && sub == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
-          v = -1;
-        }
-        const bool valid = v >= 0;
-        const uint32_t bal = __ballot_sync(0xffffffffu, valid);
-        mask |= (uint64_t)((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u)) << (4 * m);
-        const int kr = half * kChunk + r;
-        if (sub == 0 && c16 == 0) sKey[kr] = v;
-        const uint16_t* src = p.kv + (size_t)(valid ? cr : 0) * DK + c16 * 8;
-#pragma unroll
-        for (int i = 0; i < 3; ++i) {
-          const int a = sub + 3 * i;
-          uint8_t* dst = sKV + a * kAtomBytes + kr * 128 + ((c16 ^ (kr & 7)) << 4);
-          cp_async16_zfill(dst, src + a * 64, valid ? 16u : 0u);
-        }
+        // drain: the last loads of each slot land before the CTA's memory is released
+        for (int j = issued > kSlots ? issued - kSlots : 0; j < issued; ++j)
+          mbar_wait(&kv_full[(j + 2) % kSlots], (j / kSlots) & 1, p.wait_ns, no_abort);
       }
-    if (sub == 0 && lane == 0) sMask[half] = mask;
+    } else {
+    // ------------------------------------------------------------ gather: three threads per key row
+    const int r = gt / 3, part = gt - 3 * (gt / 3);     // row of the slot; 24 of its 72 chunks
+    for (int j = 0; j < nch; ++j) {
+      const int sl = (j + 2) % kSlots;
+      // slots 0 and 1 hold Q until it is in TMEM; later uses wait for the MMAs
+      if (j >= kSlots ? !wwait(&kv_empty[sl], ((j / kSlots) - 1) & 1) : (j >= 1 && !wwait(q_ready, 0))) {
+        fail(1);
+        break;
+      }
+      const int slot = j * kChunk + r;
+      int v = -1;
+      if (slot < m) v = dense ? slot : p.idx[(size_t)row * p.k + slot];
+      if (v >= Lb) {
+        if (part == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN);
+        v = -1;
+      }
+      if (v >= n) v = -1;
+      const long long cr = v >= 0 ? p.map.row(b, v) : -1;
+      if (v >= 0 && cr < 0) {
+        if (part == 0) report_error(p.err, DSA_ERR_DEVICE_BOUNDS, ERR_SITE_ATTN | (1u << 8));
+        v = -1;
+      }
+      const bool valid = v >= 0;
+      const uint16_t* src = p.kv + (size_t)(valid ? cr : 0) * DK;
+      uint8_t* dst = sKV + sl * kSlotBytes;
+#pragma unroll 4
+      for (int cc = 0; cc < 24; ++cc) {
+        const int c = part * 24 + cc;                   // 16-byte chunk of the row: atom c / 8, chunk c % 8
+        const int a = c >> 3, c16 = c & 7;
+        cp_async16_zfill(dst + a * kAtomBytes + r * 128 + ((c16 ^ (r & 7)) << 4), src + c * 8, valid ? 16u : 0u);
+      }
+      cp_async_arrive(&kv_full[sl]);
+    }
     cp_async_commit();
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    mbar_arrive(&kv_full[half]);
-    if (q_issued) mbar_wait(q_full, 0, p.wait_ns, no_abort);
+    cp_async_wait<0>();                            // every copy landed before the CTA can exit
+    }
   } else if (warp == 0) {
     // ------------------------------------------------------------ Q K^T
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(kFmtBF16, kFmtBF16, 0, 0, 128, kChunk);
-      const uint64_t kdesc0 = make_sdesc(smem_u32(sKV), 16, 1024, kSwizzle128);
-      const uint64_t qdesc0 = make_sdesc(smem_u32(sQ), 16, 1024, kSwizzle128);
-      bool ok = mbar_wait(q_full, 0, p.wait_ns, ab) && mbar_wait(q_ready, 0, p.wait_ns, ab);
-      if (!ok) fail(1);
-      int issued = 0;
-      for (int c = 0; c < 2 && ok; ++c) {
-        if (!mbar_wait(&kv_full[c], 0, p.wait_ns, ab)) { fail(2); break; }
-        fence_proxy_async_smem();
+      bool ok = mbar_wait(q_ready, 0, p.wait_ns, ab);
+      if (!ok) fail(2);
+      for (int j = 0; j < nch && ok; ++j) {
+        const int sl = (j + 2) % kSlots;
+        if (!mbar_wait(&kv_full[sl], (j / kSlots) & 1, p.wait_ns, ab)) { fail(3); ok = false; break; }
+        if (j >= 2 && !mbar_wait(&s_empty[j & 1], ((j - 2) >> 1) & 1, p.wait_ns, ab)) { fail(4); ok = false; break; }
+        fence_proxy_async_smem();                   // the gather's cp.async bytes, before the tensor core reads them
         tc_fence_after();
-        const uint32_t dS = tmem + kSCol + c * kChunk;
+        const uint32_t dS = tmem + kSCol + (j & 1) * kChunk;
+        const uint64_t kdesc0 = make_sdesc(smem_u32(sKV + sl * kSlotBytes), 16, 1024, kSwizzle128);
 #pragma unroll
         for (int ks = 0; ks < kKSteps; ++ks) {
           const int d = ks * 16;
-          const uint64_t bdesc =
-              kdesc0 + (uint64_t)(((d / 64) * kAtomBytes + (d % 64) * 2 + c * kChunk * 128) >> 4);
-          if (ks < kQTSteps) {
-            mma_bf16_ts(dS, tmem + kQCol + ks * 8, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
-          } else {
-            const int dq = d - kQT;
-            mma_bf16(dS, qdesc0 + (uint64_t)(((dq / 64) * kQAtomBytes + (dq % 64) * 2) >> 4), bdesc, idesc_qk,
-                     ks > 0 ? 1u : 0u);
-          }
+          const uint64_t bdesc = kdesc0 + (uint64_t)(((d / 64) * kAtomBytes + (d % 64) * 2) >> 4);
+          mma_bf16_ts(dS, tmem + kQCol + ks * 8, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[c]);
-        ++issued;
+        mma_commit(&s_full[j & 1]);
+        mma_commit(&kv_empty[sl]);
       }
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
-      for (int c = 0; c < issued; ++c) mbar_wait(&s_full[c], 0, p.wait_ns, no_abort);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ head sum
-    const int side = (warp - kFirstEpi) >> 2;
+    const int side = (warp - kFirstEpi) >> 2;      // key half of each chunk; dims half of Q
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const bool head_ok = h < p.H;
     {
+      // Q dims [288 side, 288 side + 288) of head h: global -> slots 0-1
+      // (own row, 16-byte chunk c of the 72 at h * 1152 + (c / 8) * 128 +
+      // ((c % 8) ^ (h % 8)) * 16) -> registers -> TMEM as BF16 pairs
       const uint16_t* qrow = p.q + ((size_t)row * p.H + (head_ok ? h : 0)) * DK;
-      for (int qb = side; qb < kQT / 64; qb += 2) {
+      uint8_t* qs = sKV + h * (DK * 2);
+#pragma unroll 4
+      for (int cc = 0; cc < 36; ++cc) {
+        const int c = side * 36 + cc;
+        cp_async16_zfill(qs + (c >> 3) * 128 + (((c & 7) ^ (h & 7)) << 4), qrow + c * 8, head_ok ? 16u : 0u);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+#pragma unroll 1
+      for (int qb = 0; qb < 5; ++qb) {
+        const int nv = qb < 4 ? 8 : 4;             // chunks of this block: 64 dims, the last 32
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           uint4 x = make_uint4(0u, 0u, 0u, 0u);
-          if (head_ok) x = *reinterpret_cast<const uint4*>(qrow + qb * 64 + i * 8);
+          const int c = side * 36 + qb * 8 + i;
+          if (i < nv) x = *reinterpret_cast<const uint4*>(qs + (c >> 3) * 128 + (((c & 7) ^ (h & 7)) << 4));
           v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
         }
-        tmem_st32(tmem + lane_addr + kQCol + qb * 32, v);
+        const uint32_t col = tmem + lane_addr + kQCol + side * (DK / 4) + qb * 32;
+        if (qb < 4) tmem_st32(col, v);
+        else tmem_st16(col, v);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -241,43 +287,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(q_ready);
     }
     const float lse2 = head_ok ? p.lse[(size_t)row * p.H + h] * 1.4426950408889634f : INFINITY;
-    bool ok = wwait(&s_full[side], 0);
-    if (!ok) fail(3);
-    if (ok && !wwait(&kv_full[side], 0)) { fail(4); ok = false; }
-    if (ok) {
-      tc_fence_after();
-      const uint64_t mask = sMask[side];
-      uint32_t s0[32], s1[32];
-      const uint32_t saddr = tmem + lane_addr + kSCol + side * kChunk;
-      tmem_ld32(saddr, s0);
-      tmem_ld32(saddr + 32, s1);
-      tmem_wait_ld_dep(s0);
-      tmem_wait_ld_dep(s1);
-      const float sc = p.scale_log2;
-      // this head's weight of each key, summed over the warp's 32 heads;
-      // lane l ends with keys l and l + 32 of this side
-      float keep0 = 0.f, keep1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const uint32_t raw = i < 32 ? s0[i] : s1[i - 32];
-        float e = head_ok ? exp2f(fmaf(__uint_as_float(raw), sc, -lse2)) : 0.f;
-        if (!((mask >> i) & 1ull)) e = 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-        if (i == lane) keep0 = e;
-        if (i == lane + 32) keep1 = e;
+    const float sc = p.scale_log2;
+    const float inv_h = 1.0f / (float)p.H;
+    float* target = p.target + (size_t)lr * p.ld;
+    // every warp takes every iteration (a failed wait only skips the work),
+    // so the named barriers below always fill
+    bool ok = true;
+    for (int j = 0; j < nch; ++j) {
+      float part = 0.f;
+      if (ok && !wwait(&s_full[j & 1], (j >> 1) & 1)) {
+        fail(5);
+        ok = false;
       }
-      atomicAdd(&sSum[side * 64 + lane], keep0);
-      atomicAdd(&sSum[side * 64 + lane + 32], keep1);
-    }
-    // the eight head-sum warps meet, then write this split's keys
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-    if (ok) {
-      const int i = threadIdx.x - kFirstEpi * 32;          // 0..255: slots i < 128 write
-      if (i < kKeys && ((sMask[i >> 6] >> (i & 63)) & 1ull)) {
-        const int key = sKey[i];
-        const long long o = (long long)lr * p.ld + key;
-        if (key >= 0 && key < p.ld) p.target[o] = sSum[i] / (float)p.H;
+      if (ok) {
+        tc_fence_after();
+        uint32_t s[32];
+        tmem_ld32(tmem + lane_addr + kSCol + (j & 1) * kChunk + side * 32, s);
+        tmem_wait_ld_dep(s);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[j & 1]);
+        float e[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) e[i] = exp2f(fmaf(__uint_as_float(s[i]), sc, -lse2));
+        part = transpose_reduce32(e, lane);          // this warp's 32 heads, key side * 32 + lane
+      }
+      float* sum = sSum + (j & 1) * kChunk + side * 32 + lane;
+      if (ok) atomicAdd(sum, part);
+      // the four quarters of this key half meet; quarter 0 writes the keys
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + side), "n"(128) : "memory");
+      if (quarter == 0) {
+        // the key of this slot, as the gather read it
+        const int slot = j * kChunk + side * 32 + lane;
+        int key = -1;
+        if (slot < m) key = dense ? slot : p.idx[(size_t)row * p.k + slot];
+        if (key >= n || (key >= 0 && p.map.row(b, key) < 0)) key = -1;
+        if (ok && key >= 0) target[key] = *sum * inv_h;
+        *sum = 0.f;
       }
     }
   }
@@ -530,19 +576,18 @@ extern "C" dsa_status dsa_kl_target(const dsa_shape* s, const uint16_t* q, const
   p.map = api_kv_map(s);
   p.q = q; p.kv = kv; p.lse = lse; p.idx = idx; p.target = target; p.ld = ld;
   p.T = s->T; p.H = s->H; p.k = s->k; p.q_begin = q_begin; p.q_count = q_count; p.B = s->B;
-  const int slots = idx ? s->k : s->S;
-  p.nsplit = (slots + kKeys - 1) / kKeys;
   const float tau = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / sqrtf((float)s->d_k);
   p.scale_log2 = tau * 1.4426950408889634f;
   p.wait_ns = c.wait_ns;
   p.err = c.err;
-  CUtensorMap tm_q;
-  if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, (uint64_t)s->B * s->T * s->H, DK, (uint64_t)DK * 2,
-                    128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  CUtensorMap tm_kv = {};
+  p.tma_keys = idx == nullptr && p.map.page_size == 0;
+  if (p.tma_keys && !make_tmap_2d(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, (uint64_t)s->B * s->S, DK,
+                                  (uint64_t)DK * 2, kChunk, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   if (cudaFuncSetAttribute(kl_target_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return DSA_ERR_CUDA;
-  kl_target_kernel<<<(unsigned)((long long)s->B * q_count * p.nsplit), kThreads, kSmem, c.stream>>>(tm_q, p);
+  kl_target_kernel<<<(unsigned)((long long)s->B * q_count), kThreads, kSmem, c.stream>>>(tm_kv, p);
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
