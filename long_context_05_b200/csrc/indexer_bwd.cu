@@ -27,10 +27,11 @@
 // The hi + lo splits keep about 16 bits of every FP32 factor, so the
 // gradients carry FP32-like error although the tensor cores read BF16.
 //
-// Warp roles (416 threads, one query row per CTA): warp 0 issues the MMAs;
-// warps 1-4 gather the tile's key rows (k_I bytes, by cp.async) and per-key
-// scalars into a 4-stage ring; warps 5-12 read D^T from TMEM, build P, G^T
-// and K16 in shared memory, and add each tile's dk into global memory.
+// Warp roles (672 threads, one query row per CTA): warp 0 issues the MMAs;
+// warps 1-4 gather the tile's key rows (k_I bytes, by cp.async) and g_s ks_s
+// into a 3-stage ring; warps 5-12 read D^T from TMEM and build P, G^T and K16
+// in shared memory (and finish dq, dw at the row's end); warps 13-20 add each
+// tile's dk into global memory while the next tile is being built.
 #include <cuda_fp8.h>
 #include <math.h>
 
@@ -46,9 +47,9 @@ namespace ib {
 constexpr int kKeys = 128;      // keys per tile: TMEM lanes of D^T and dk
 constexpr int kHeads = 64;      // indexer heads, zero-padded up to 64
 constexpr int kDim = 128;       // D_I
-constexpr int kStages = 4;      // key-row ring
-constexpr int kFirstGather = 1, kGatherWarps = 4, kFirstEpi = 5, kEpiWarps = 8;
-constexpr int kThreads = 32 * (kFirstEpi + kEpiWarps);
+constexpr int kStages = 3;      // key-row ring
+constexpr int kFirstGather = 1, kGatherWarps = 4, kFirstEpi = 5, kEpiWarps = 8, kFirstRd = 13, kRdWarps = 8;
+constexpr int kThreads = 32 * (kFirstRd + kRdWarps);
 constexpr int kK8Bytes = kKeys * 128;                       // FP8 key rows, 128B-swizzled K-major
 constexpr int OFF_K8 = 0;
 constexpr int OFF_GT = OFF_K8 + kStages * kK8Bytes;         // G^T: 2 atoms (keys 0-63, 64-127) of 128 rows x 128 B
@@ -57,12 +58,12 @@ constexpr int OFF_P = OFF_K16 + 2 * 128 * 128;              // P: 128 keys x 64 
 constexpr int OFF_Q8 = OFF_P + 128 * 128;                   // Q8: 64 heads x 128 B
 constexpr int OFF_QH = OFF_Q8 + kHeads * 128;               // Q'hi: 2 atoms (dims) of 64 heads x 128 B
 constexpr int OFF_QL = OFF_QH + 2 * kHeads * 128;           // Q'lo
-constexpr int OFF_ROW = OFF_QL + 2 * kHeads * 128;          // per stage: cache row of each key (int, -1: none)
-constexpr int OFF_G = OFF_ROW + kStages * kKeys * 4;        // per stage: g_s
-constexpr int OFF_C = OFF_G + kStages * kKeys * 4;          // per stage: g_s ks_s
+constexpr int OFF_C = OFF_QL + 2 * kHeads * 128;            // per stage: g_s ks_s of each key
 constexpr int OFF_HEAD = OFF_C + kStages * kKeys * 4;       // w[64], qs[64], dw halves [2][64]
-constexpr int OFF_BAR = OFF_HEAD + 4 * kHeads * 4;
-// q_full, k8_full[4], k8_empty[4], d_full[2], d_empty[2], p_full, p_empty,
+constexpr int kStageStride = 144;                           // dk staging: 32 floats per key + 16 B pad
+constexpr int OFF_STAGE = OFF_HEAD + 4 * kHeads * 4;        // per dk reader warp: 32 keys x kStageStride
+constexpr int OFF_BAR = OFF_STAGE + kRdWarps * 32 * kStageStride;
+// q_full, k8_full[3], k8_empty[3], d_full[2], d_empty[2], p_full, p_empty,
 // dk_full[2], dk_empty[2], mma_done
 constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 2 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
@@ -141,8 +142,6 @@ __global__ void __launch_bounds__(ib::kThreads, 1) indexer_bwd_tc_kernel(BwdPara
   uint8_t* sQ8 = smem + OFF_Q8;
   uint8_t* sQH = smem + OFF_QH;
   uint8_t* sQL = smem + OFF_QL;
-  int* sRow = reinterpret_cast<int*>(smem + OFF_ROW);
-  float* sG = reinterpret_cast<float*>(smem + OFF_G);
   float* sC = reinterpret_cast<float*>(smem + OFF_C);
   float* sW = reinterpret_cast<float*>(smem + OFF_HEAD);
   float* sQs = sW + kHeads;
@@ -180,7 +179,7 @@ __global__ void __launch_bounds__(ib::kThreads, 1) indexer_bwd_tc_kernel(BwdPara
       mbar_init(&d_full[i], 1);
       mbar_init(&d_empty[i], kEpiWarps);
       mbar_init(&dk_full[i], 1);
-      mbar_init(&dk_empty[i], kEpiWarps);
+      mbar_init(&dk_empty[i], kRdWarps);
     }
     mbar_init(p_full, kEpiWarps);
     mbar_init(p_empty, 1);
@@ -227,8 +226,6 @@ __global__ void __launch_bounds__(ib::kThreads, 1) indexer_bwd_tc_kernel(BwdPara
       const bool valid = row >= 0;
       const float g = valid ? G[s] : 0.f;
       const float ks = valid ? p.k_scale[row] : 0.f;
-      sRow[st * kKeys + kk] = valid ? (int)row : -1;
-      sG[st * kKeys + kk] = g;
       sC[st * kKeys + kk] = g * ks;
       const uint8_t* src = p.k_I + (size_t)(valid ? row : 0) * kDim;
       uint8_t* dst = sK8 + st * kK8Bytes;
@@ -310,6 +307,70 @@ __global__ void __launch_bounds__(ib::kThreads, 1) indexer_bwd_tc_kernel(BwdPara
       mbar_wait(mma_done, 0, p.wait_ns, no_abort);
     }
     __syncwarp();
+  } else if (warp >= kFirstRd) {
+    // ------------------------------------------------------------ dk reader
+    // dk of each tile: TMEM -> registers, times g_s, through this warp's
+    // staging rows so that each red.v4 of the warp covers four keys' 128
+    // contiguous bytes (8 rounds for the warp's 32 keys), added into dk
+    // (global).  The key's cache row and g_s are read again from global
+    // memory (before the wait), so nothing is shared with the other roles.
+    const int h = (warp - kFirstRd) >> 2;          // dims 64h .. 64h + 63
+    const int q = warp & 3;
+    const int sl = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    uint8_t* stage = smem + OFF_STAGE + (warp - kFirstRd) * 32 * kStageStride;
+    const float* G = p.grad + (size_t)lr * p.ld;
+    for (int i = 0; i < nt; ++i) {
+      const int slot = i * kKeys + sl;
+      int s = -1;
+      if (slot < m) s = set ? set[slot] : slot;
+      int row = -1;
+      float g = 0.f;
+      if (s >= 0 && s < n) {
+        const long long r = p.map.row(b, s);
+        if (r >= 0) {
+          row = (int)r;
+          g = G[s];
+        }
+      }
+      if (!wwait(&dk_full[i & 1], (i >> 1) & 1)) {
+        fail(7);
+        break;
+      }
+      tc_fence_after();
+      uint32_t a[2][32];
+      const uint32_t col = tmem + lane_addr + kColDk + (i & 1) * kDim + h * 64;
+      tmem_ld32(col, a[0]);
+      tmem_ld32(col + 32, a[1]);
+      tmem_wait_ld_dep(a[0]);
+      tmem_wait_ld_dep(a[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dk_empty[i & 1]);
+      const float gs = row >= 0 ? g : 0.f;
+#pragma unroll
+      for (int ps = 0; ps < 2; ++ps) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(stage + lane * kStageStride + c * 16, __float_as_uint(gs * __uint_as_float(a[ps][4 * c])),
+                       __float_as_uint(gs * __uint_as_float(a[ps][4 * c + 1])),
+                       __float_as_uint(gs * __uint_as_float(a[ps][4 * c + 2])),
+                       __float_as_uint(gs * __uint_as_float(a[ps][4 * c + 3])));
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int kl = it * 4 + (lane >> 3), c = lane & 7;   // key of the warp, float4 of its 32 floats
+          const int rw = __shfl_sync(0xffffffffu, row, kl);
+          const float gk = __shfl_sync(0xffffffffu, gs, kl);
+          const uint4 v = ld_shared_v4(stage + kl * kStageStride + c * 16);
+          if (rw >= 0 && gk != 0.f)
+            atomicAdd(reinterpret_cast<float4*>(p.dk + (size_t)rw * kDim + h * 64 + ps * 32 + c * 4),
+                      make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                                  __uint_as_float(v.w)));
+        }
+        __syncwarp();
+      }
+    }
   } else if (warp >= kFirstEpi) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - kFirstEpi;
@@ -356,44 +417,9 @@ __global__ void __launch_bounds__(ib::kThreads, 1) indexer_bwd_tc_kernel(BwdPara
       fence_proxy_async_smem();
       mbar_arrive(q_full);
     }
-    float g_prev = 0.f;
-    int row_prev = -1;
-    // dk of tile jt: TMEM -> registers, times g_s, added into dk (global)
-    auto readout = [&](int jt) -> bool {
-      if (!wwait(&dk_full[jt & 1], (jt >> 1) & 1)) {
-        fail(7);
-        return false;
-      }
-      tc_fence_after();
-      uint32_t a[32], c[32];
-      const uint32_t col = tmem + lane_addr + kColDk + (jt & 1) * kDim + h * 64;
-      tmem_ld32(col, a);
-      tmem_ld32(col + 32, c);
-      tmem_wait_ld_dep(a);
-      tmem_wait_ld_dep(c);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&dk_empty[jt & 1]);
-      if (row_prev >= 0 && g_prev != 0.f) {
-        float4* dst = reinterpret_cast<float4*>(p.dk + (size_t)row_prev * kDim + h * 64);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          atomicAdd(dst + v, make_float4(g_prev * __uint_as_float(a[4 * v]), g_prev * __uint_as_float(a[4 * v + 1]),
-                                         g_prev * __uint_as_float(a[4 * v + 2]),
-                                         g_prev * __uint_as_float(a[4 * v + 3])));
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          atomicAdd(dst + 8 + v,
-                    make_float4(g_prev * __uint_as_float(c[4 * v]), g_prev * __uint_as_float(c[4 * v + 1]),
-                                g_prev * __uint_as_float(c[4 * v + 2]), g_prev * __uint_as_float(c[4 * v + 3])));
-      }
-      return true;
-    };
     for (int i = 0; i < nt && ok; ++i) {
       const int st = i % kStages;
       if (!wwait(&k8_full[st], (i / kStages) & 1)) { fail(8); ok = false; break; }
-      const float g_cur = sG[st * kKeys + sl];
-      const int row_cur = sRow[st * kKeys + sl];
       if (!wwait(&d_full[i & 1], (i >> 1) & 1)) { fail(9); ok = false; break; }
       tc_fence_after();
       uint32_t r[32];
@@ -469,11 +495,7 @@ __global__ void __launch_bounds__(ib::kThreads, 1) indexer_bwd_tc_kernel(BwdPara
         mbar_arrive(p_full);
         mbar_arrive(&k8_empty[st]);
       }
-      if (i >= 1 && !readout(i - 1)) { ok = false; break; }
-      g_prev = g_cur;
-      row_prev = row_cur;
     }
-    if (ok && nt >= 1 && !readout(nt - 1)) ok = false;
     // R: lo rows (lanes 64..127) through shared memory onto the hi rows
     if (ok && nt >= 1 && !wwait(p_empty, (nt - 1) & 1)) { fail(11); ok = false; }
     float* X = reinterpret_cast<float*>(sK16);           // [64][132]
