@@ -88,9 +88,6 @@ def measured_traffic(workload: str, kernel: str):
     return t["bytes"]
 FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# FP32 FMA issue on CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
-# (clocks.max.sm); the peak of kernels that run plain FP32 arithmetic
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
 
 
 # ------------------------------------------------------------------ helpers
@@ -782,10 +779,14 @@ def extra_train(wl, steps, warmup, ws, peaks, peak_src):
                                      bf16, f"bf16 sustained ({peak_src}); Q K^T of the set"),
             "indexer_kl": part_report(per["indexer_kl"], kl_bytes / 1e9, "GB/s", "hbm", peaks["hbm_gbs"],
                                       f"hbm ({peak_src}); scores + target of the set read, grad row written"),
+            # tensor cores (D in FP8, dk and R in BF16 hi + lo); algorithmic
+            # FLOP: D, dq and dk per pair.  Its dk additions into global
+            # memory (512 B per pair) are reported beside it
             "indexer_backward": part_report(per["indexer_backward"], 6.0 * wl.H_I * wl.D_I * pairs / 1e12,
-                                            "TFLOP/s", "alu", FP32_ALU_TFLOPS,
-                                            "fp32 FMA, 148 SMs x 128 lanes at 1965 MHz; D, dq and dk per pair"),
+                                            "TFLOP/s", "tensor", bf16,
+                                            f"bf16 sustained ({peak_src}); D, dq and dk per pair"),
         }
+        parts["indexer_backward"]["dk_reduce_gbs"] = 4.0 * wl.D_I * pairs / (per["indexer_backward"] / 1e3) / 1e9
         res[stage] = {"ms_per_step": ms, "rows_per_s": ws * wl.B * wl.T / (ms / 1e3), "gpu_launches": launches,
                       "kernels": parts}
     st, det = dsa.device_error()
