@@ -40,11 +40,11 @@ namespace {
 using namespace sm100;
 
 constexpr int kBM = 128;       // keys per tile (MMA M)
-constexpr int kNSub = 128;     // MMA N: (query, head) rows per sub-tile
+constexpr int kNSub = 128;     // MMA N: (query, head) rows per sub-tile (64 in the one-query form)
 constexpr int kMaxNB = 8;      // sub-tiles per work item
 constexpr int kKC = 32;        // key tiles per work item (at most; fewer when items are scarce)
 constexpr int kStages = 4;     // depth of the k_I ring
-constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * kNSub = 512 columns)
+constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * NS columns)
 static_assert((kNAcc & (kNAcc - 1)) == 0, "accumulator index is taken with a mask");
 // Key tiles per accumulator group: with many heads (HI >= 32) two
 // consecutive key tiles share one pass of the epilogue over a sub-tile, so
@@ -84,16 +84,16 @@ struct IdxParams {
   DevErr* err;
 };
 
-template <int DI>
+template <int DI, int NS>
 struct Layout {
   static constexpr int kABytes = kBM * DI;
-  static constexpr int kBSubBytes = kNSub * DI;
+  static constexpr int kBSubBytes = NS * DI;
   static constexpr int kBOff = 0;
   static constexpr int kAOff = kBOff + kMaxNB * kBSubBytes;
   static constexpr int kWOff = kAOff + kStages * kABytes;            // wM, two item buffers
-  static constexpr int kWFloats = kMaxNB * kNSub;
+  static constexpr int kWFloats = kMaxNB * NS;
   static constexpr int kThrOff = kWOff + 2 * kWFloats * 4;           // thresholds, two item buffers
-  static constexpr int kThrWords = kMaxNB * kNSub / 4;               // queries per item at most (4 heads)
+  static constexpr int kThrWords = kMaxNB * NS / 4;                  // queries per item at most (4 heads)
   static constexpr int kBarOff = kThrOff + 2 * kThrWords * 4;
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNAcc + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
@@ -111,11 +111,11 @@ struct Item {
   int off;  // L - T: pos(t) = off + t
 };
 
-template <int HI, bool PLAIN, class F>
+template <int HI, int NS, bool PLAIN, class F>
 __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
   const int KS = PLAIN ? 1 : p.kstride;
   const int* const SLOT = PLAIN ? nullptr : p.row_slot;
-  constexpr int QPS = kNSub / HI;
+  constexpr int QPS = NS / HI;
   const int per_group = p.nb * QPS;
   const int grid = gridDim.x, cta = blockIdx.x;
   long long flat = 0;
@@ -153,14 +153,14 @@ __device__ __forceinline__ void for_each_item(const IdxParams& p, F&& f) {
 // the active sub-tiles (some query sees a key of the tile) are [jlo, nsub):
 // the last query of sub-tile j grows with j, and the item's last query sees
 // every key tile the item covers.
-template <int HI>
+template <int HI, int NS>
 __device__ __forceinline__ int item_nsub(const IdxParams& p, const Item& it) {
-  constexpr int QPS = kNSub / HI;
+  constexpr int QPS = NS / HI;
   return min(p.nb, (it.tend - it.t0 + QPS - 1) / QPS);
 }
-template <int HI, bool PLAIN>
+template <int HI, int NS, bool PLAIN>
 __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, int kt, int nsub) {
-  constexpr int QPS = kNSub / HI;
+  constexpr int QPS = NS / HI;
   // smallest j with t0 + (j + 1) * QPS - 1 >= kt * kBM * kstride - off
   const int x = kt * kBM * (PLAIN ? 1 : p.kstride) - it.off - it.t0 + QPS;
   const int j = x > 0 ? x / QPS - 1 : 0;
@@ -173,12 +173,14 @@ __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, 
 // candidate and the repair modes, whose checks the plain form must not pay.
 // CAND: candidate mode (thr set).  With PLAIN it keeps the contiguous
 // fast paths while appending candidates instead of storing scores.
-template <int DI, int HI, bool PLAIN, bool CAND>
+// NS: MMA N, the (query, head) rows of a sub-tile: 128, or 64 where every
+// sequence has one query (decode), so that no half of a sub-tile is padding.
+template <int DI, int HI, bool PLAIN, bool CAND, int NS>
 __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                       IdxParams p) {
-  using L = Layout<DI>;
-  constexpr int QPS = kNSub / HI;
+  using L = Layout<DI, NS>;
+  constexpr int QPS = NS / HI;
   // the plain form sees constants: no sample stride, no candidates, no repair
   const int KS = PLAIN ? 1 : p.kstride;
   const unsigned int* const THR = CAND ? p.thr : nullptr;
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kNAcc * kNSub);
+    tmem_alloc(tmem_slot, kNAcc * NS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       bool issued[kStages];
       for (int i = 0; i < kStages; ++i) issued[i] = false;
       bool ok = true;
-      for_each_item<HI, PLAIN>(p, [&](const Item& it) {
+      for_each_item<HI, NS, PLAIN>(p, [&](const Item& it) {
         const int bb = nbbuf == 2 ? (int)(items & 1) : 0;
         const uint32_t use = nbbuf == 2 ? items >> 1 : items;
         if (!mbar_wait(&b_empty[bb], (use & 1) ^ 1, p.wait_ns, ab)) { fail(1); ok = false; return false; }
@@ -312,19 +314,19 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc(kFmtE4M3, kFmtE4M3, 0, 0, kBM, kNSub);
+      constexpr uint32_t idesc = make_idesc(kFmtE4M3, kFmtE4M3, 0, 0, kBM, NS);
       using E = EpiCfg<HI>;
       uint32_t a_cnt = 0, items = 0, u = 0;
       // descriptors built once; a stage or sub-tile only adds its offset >> 4
       const uint64_t adesc0 = make_sdesc(smem_u32(sA), 16, L::kSBO, L::kSwizzleLayout);
       const uint64_t bdesc0 = make_sdesc(smem_u32(sB), 16, L::kSBO, L::kSwizzleLayout);
-      for_each_item<HI, PLAIN>(p, [&](const Item& it) {
+      for_each_item<HI, NS, PLAIN>(p, [&](const Item& it) {
         const int bb = nbbuf == 2 ? (int)(items & 1) : 0;
         const uint32_t use = nbbuf == 2 ? items >> 1 : items;
         if (!mbar_wait(&b_full[bb], use & 1, p.wait_ns, ab)) { fail(3); return false; }
         ++items;
         const uint64_t bdesc_it = bdesc0 + (uint64_t)((bb * kBBufBytes) >> 4);
-        const int nsub = item_nsub<HI>(p, it);
+        const int nsub = item_nsub<HI, NS>(p, it);
         const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
         for (int kt = kt0; kt < kt1; kt += E::G) {
           // key tiles kt .. kt + ng - 1 of this group, each in its ring stage
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           tc_fence_after();
           // the first active sub-tile of kt also covers kt + 1 (later keys
           // need later queries); masked pairs are computed and dropped
-          for (int j = first_active<HI, PLAIN>(p, it, kt, nsub); j < nsub; ++j) {
+          for (int j = first_active<HI, NS, PLAIN>(p, it, kt, nsub); j < nsub; ++j) {
             const int slot = u % E::NSLOT;
             if (!mbar_test_wait(&acc_empty[slot], ((u / E::NSLOT) & 1) ^ 1) &&
                 !mbar_wait(&acc_empty[slot], ((u / E::NSLOT) & 1) ^ 1, p.wait_ns, ab)) {
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
 #pragma unroll
             for (int g = 0; g < E::G; ++g) {
               if (g >= ng) break;
-              const uint32_t dacc = tmem_base + (slot * E::G + g) * kNSub;
+              const uint32_t dacc = tmem_base + (slot * E::G + g) * NS;
 #pragma unroll
               for (int ks = 0; ks < DI / 32; ++ks)
                 mma_f8(dacc, adesc[g] + 2 * ks, bdesc + 2 * ks, idesc, ks > 0 ? 1u : 0u);
@@ -386,10 +388,10 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     // candidate mode: this warp's list and its length (warp-uniform)
     const long long wl0 = ((long long)blockIdx.x * (E::EPI_THREADS / 32) + ew) * p.wl_cap;
     long long wpos = 0;
-    for_each_item<HI, PLAIN>(p, [&](const Item& it) {
+    for_each_item<HI, NS, PLAIN>(p, [&](const Item& it) {
       // per-item head weights  wM[(query, head)] = w * q_scale  (0 past the end)
       float* wbuf = sW + (items & 1) * L::kWFloats;
-      for (int x = etid; x < p.nb * kNSub; x += E::EPI_THREADS) {
+      for (int x = etid; x < p.nb * NS; x += E::EPI_THREADS) {
         const int t = it.t0 + x / HI;
         float v = 0.f;
         if (t < it.tend) {
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       if (!mbar_wait(&w_ready[items & 1], (items >> 1) & 1, p.wait_ns, ab)) { fail(7); return false; }
       const unsigned int* tq = sThr + (items & 1) * L::kThrWords;
       ++items;
-      const int nsub = item_nsub<HI>(p, it);
+      const int nsub = item_nsub<HI, NS>(p, it);
       const int kt0 = it.c * p.kc, kt1 = min(kt0 + p.kc, it.ntiles);
       for (int kt = kt0; kt < kt1; kt += E::G) {
         const int ng = min(E::G, kt1 - kt);
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
             ksg[g] = kr >= 0 ? 0.5f * p.k_scale[kr] : 0.f;
           }
         }
-        const int jlo = first_active<HI, PLAIN>(p, it, kt, nsub);
+        const int jlo = first_active<HI, NS, PLAIN>(p, it, kt, nsub);
         const uint32_t u0 = u;
         u += (uint32_t)(nsub - jlo);
         // this group's sub-tiles: my = u0 + (j - jlo) == grp (mod NGRP)
@@ -438,8 +440,8 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
           const bool got = mbar_wait(&acc_full[slot], (my / E::NSLOT) & 1, p.wait_ns, ab);
           if (!__all_sync(0xffffffffu, got)) { fail(6); return false; }
           tc_fence_after();
-          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot * E::G * kNSub;
-          const float* wq = wbuf + j * kNSub;
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + slot * E::G * NS;
+          const float* wq = wbuf + j * NS;
           // w * ReLU(x) summed over the heads of each query, for each key tile
           // of the group; four independent packed-pair partial sums per
           // (tile, query) keep the FMA chains short.  ReLU is formed as
@@ -457,14 +459,14 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
               for (int i = 0; i < NP; ++i) part[g][q][i] = make_float2(0.f, 0.f);
           uint32_t v[2][E::G][CW];
 #pragma unroll
-          for (int g = 0; g < E::G; ++g) tmem_ld16(taddr + g * kNSub, v[0][g]);
+          for (int g = 0; g < E::G; ++g) tmem_ld16(taddr + g * NS, v[0][g]);
 #pragma unroll
           for (int g = 0; g < E::G; ++g) tmem_wait_ld_dep(v[0][g]);
 #pragma unroll
-          for (int c = 0; c < kNSub / CW; ++c) {
-            if (c + 1 < kNSub / CW) {
+          for (int c = 0; c < NS / CW; ++c) {
+            if (c + 1 < NS / CW) {
 #pragma unroll
-              for (int g = 0; g < E::G; ++g) tmem_ld16(taddr + g * kNSub + (c + 1) * CW, v[(c + 1) & 1][g]);
+              for (int g = 0; g < E::G; ++g) tmem_ld16(taddr + g * NS + (c + 1) * CW, v[(c + 1) & 1][g]);
             } else {
               // every column of the group's accumulators is in registers
               tc_fence_before();
@@ -489,7 +491,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
                 }
               }
             }
-            if (c + 1 < kNSub / CW) {
+            if (c + 1 < NS / CW) {
 #pragma unroll
               for (int g = 0; g < E::G; ++g) tmem_wait_ld_dep(v[(c + 1) & 1][g]);
             }
@@ -565,14 +567,14 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kNAcc * kNSub);
+    tmem_dealloc(tmem_base, kNAcc * NS);
   }
 }
 
-template <int DI, int HI>
+template <int DI, int HI, int NS>
 cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
-  using L = Layout<DI>;
-  constexpr int QPS = kNSub / HI;
+  using L = Layout<DI, NS>;
+  constexpr int QPS = NS / HI;
   CUtensorMap tm_k, tm_q;
   const CUtensorMapSwizzle sw = DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : DI == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -591,7 +593,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   if (!make_tmap_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.k_I, (uint64_t)(pool_rows / ks), DI,
                     (uint64_t)DI * ks, box_rows, DI, sw))
     return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_I, (uint64_t)a.B * a.T * HI, DI, DI, kNSub, DI, sw))
+  if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.q_I, (uint64_t)a.B * a.T * HI, DI, DI, NS, DI, sw))
     return cudaErrorInvalidValue;
   IdxParams p = {};
   p.kv = a.kv;
@@ -657,8 +659,9 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   // list), with score rows or candidate lists as the output
   const bool plain = ks == 1 && p.row_slot == nullptr && a.kv.page_size == 0 && a.kv.seqlens == nullptr;
   const bool cand = p.thr != nullptr;
-  auto kern = cand ? (plain ? indexer_tc_kernel<DI, HI, true, true> : indexer_tc_kernel<DI, HI, false, true>)
-                   : (plain ? indexer_tc_kernel<DI, HI, true, false> : indexer_tc_kernel<DI, HI, false, false>);
+  auto kern = cand ? (plain ? indexer_tc_kernel<DI, HI, true, true, NS> : indexer_tc_kernel<DI, HI, false, true, NS>)
+                   : (plain ? indexer_tc_kernel<DI, HI, true, false, NS>
+                            : indexer_tc_kernel<DI, HI, false, false, NS>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   kern<<<grid, EpiCfg<HI>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
@@ -669,11 +672,12 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
 template <int DI>
 cudaError_t launch_di(const LaunchCtx& c, const IndexerArgs& a) {
   switch (a.H_I) {
-    case 4: return launch_tc<DI, 4>(c, a);
-    case 8: return launch_tc<DI, 8>(c, a);
-    case 16: return launch_tc<DI, 16>(c, a);
-    case 32: return launch_tc<DI, 32>(c, a);
-    case 64: return launch_tc<DI, 64>(c, a);
+    case 4: return launch_tc<DI, 4, kNSub>(c, a);
+    case 8: return launch_tc<DI, 8, kNSub>(c, a);
+    case 16: return launch_tc<DI, 16, kNSub>(c, a);
+    case 32: return launch_tc<DI, 32, kNSub>(c, a);
+    // one query per sequence (decode): sub-tiles of one query's 64 heads
+    case 64: return a.q_count == 1 ? launch_tc<DI, 64, 64>(c, a) : launch_tc<DI, 64, kNSub>(c, a);
     default: return cudaErrorInvalidValue;
   }
 }
