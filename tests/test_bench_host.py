@@ -71,3 +71,30 @@ def test_traffic_reported_only_for_the_captured_source(bench):
     assert got == (t["bytes"] if same else None)
     assert bench.measured_traffic("prefill_8k", "sparse_attn") is None
     assert bench.measured_traffic("prefill_128k", "indexer") is None
+
+
+def test_paged_layout_places_every_token():
+    """to_paged (the paged caches of the tests and the bench's paged decode):
+    token s of sequence b lands at pool row table[b, s // P] * P + s % P with
+    every key-side array moved alike, no two tokens share a pool row, the
+    table's extra column is -1, and the spare pool pages stay zero."""
+    import torch
+    from long_context_05_b200.inputs import Workload, make_inputs, to_paged
+    wl = Workload("paged_host", B=3, T=1, S=1000, H_I=4, D_I=32, H=8, d_k=80, d_v=64, k=64, q_block=1, seed=21)
+    inp = make_inputs(wl, "cpu")
+    inp["v"] = torch.randn(wl.B, wl.S, wl.d_v).to(torch.bfloat16)
+    P = 64
+    pin, table, num_pages = to_paged(inp, wl, P, 22)
+    ppseq = (wl.S + P - 1) // P
+    assert num_pages == wl.B * ppseq + 2 and tuple(table.shape) == (wl.B, ppseq + 1)
+    t = table.numpy()
+    assert (t[:, -1] == -1).all()
+    assert sorted(t[:, :ppseq].ravel().tolist()) == sorted(set(t[:, :ppseq].ravel().tolist()))
+    s = torch.arange(wl.S)
+    for b in range(wl.B):
+        rows = torch.from_numpy(t[b, (s // P).numpy()]).long() * P + s % P
+        for name in ("k_I", "k_scale", "kv", "v"):
+            assert torch.equal(pin[name][rows], inp[name][b]), (name, b)
+    used = set(t[:, :ppseq].ravel().tolist())
+    for pg in set(range(num_pages)) - used:
+        assert not pin["kv"][pg * P:(pg + 1) * P].float().abs().any()
