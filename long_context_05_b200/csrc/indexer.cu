@@ -41,21 +41,23 @@ using namespace sm100;
 
 constexpr int kBM = 128;       // keys per tile (MMA M)
 constexpr int kNSub = 128;     // MMA N: (query, head) rows per sub-tile (64 in the one-query form)
-constexpr int kMaxNB = 8;      // sub-tiles per work item
 constexpr int kKC = 32;        // key tiles per work item (at most; fewer when items are scarce)
 constexpr int kStages = 4;     // depth of the k_I ring
 constexpr int kNAcc = 4;       // TMEM accumulators (kNAcc * NS columns)
 static_assert((kNAcc & (kNAcc - 1)) == 0, "accumulator index is taken with a mask");
 // Key tiles per accumulator group: with many heads (HI >= 32) two
 // consecutive key tiles share one pass of the epilogue over a sub-tile, so
-// every head-weight load from shared memory serves two accumulators.
-template <int HI>
+// every head-weight load from shared memory serves two accumulators.  The
+// one-query form (NS = 64) runs one epilogue group and a small shared
+// memory layout, so that two CTAs (two MMA-issuing threads) share an SM.
+template <int HI, int NS>
 struct EpiCfg {
-  static constexpr int G = HI >= 32 ? 2 : 1;       // key tiles per group
-  static constexpr int NSLOT = kNAcc / G;          // accumulator groups in flight
-  static constexpr int NGRP = G == 2 ? 2 : 3;      // epilogue groups of four warps
+  static constexpr int G = HI >= 32 ? 2 : 1;                     // key tiles per group
+  static constexpr int NSLOT = kNAcc / G;                        // accumulator groups in flight
+  static constexpr int NGRP = NS == 64 ? 1 : (G == 2 ? 2 : 3);   // epilogue groups of four warps
   static constexpr int EPI_THREADS = 128 * NGRP;
   static constexpr int THREADS = 64 + EPI_THREADS;
+  static constexpr int CTAS_PER_SM = NS == 64 ? 2 : 1;
 };
 
 struct IdxParams {
@@ -86,6 +88,7 @@ struct IdxParams {
 
 template <int DI, int NS>
 struct Layout {
+  static constexpr int kMaxNB = NS == 64 ? 2 : 8;   // sub-tiles per work item
   static constexpr int kABytes = kBM * DI;
   static constexpr int kBSubBytes = NS * DI;
   static constexpr int kBOff = 0;
@@ -176,7 +179,7 @@ __device__ __forceinline__ int first_active(const IdxParams& p, const Item& it, 
 // NS: MMA N, the (query, head) rows of a sub-tile: 128, or 64 where every
 // sequence has one query (decode), so that no half of a sub-tile is padding.
 template <int DI, int HI, bool PLAIN, bool CAND, int NS>
-__global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
+__global__ void __launch_bounds__(EpiCfg<HI, NS>::THREADS, EpiCfg<HI, NS>::CTAS_PER_SM)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                       IdxParams p) {
   using L = Layout<DI, NS>;
@@ -210,8 +213,8 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
   // With at most half of the B sub-tiles in use (few queries per item, as in
   // decode), the B region holds two item buffers, so the next item's B and
   // its first key tiles load while the current item's MMAs run.
-  const int nbbuf = p.nb * 2 <= kMaxNB ? 2 : 1;
-  constexpr int kBBufBytes = kMaxNB / 2 * L::kBSubBytes;
+  const int nbbuf = p.nb * 2 <= L::kMaxNB ? 2 : 1;
+  constexpr int kBBufBytes = L::kMaxNB / 2 * L::kBSubBytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -227,8 +230,8 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
       mbar_init(&acc_empty[i], 4);  // one arrive per epilogue warp of the owning group
     }
     mbar_init(mma_done, 1);
-    mbar_init(&w_ready[0], EpiCfg<HI>::EPI_THREADS);
-    mbar_init(&w_ready[1], EpiCfg<HI>::EPI_THREADS);
+    mbar_init(&w_ready[0], EpiCfg<HI, NS>::EPI_THREADS);
+    mbar_init(&w_ready[1], EpiCfg<HI, NS>::EPI_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -315,7 +318,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc(kFmtE4M3, kFmtE4M3, 0, 0, kBM, NS);
-      using E = EpiCfg<HI>;
+      using E = EpiCfg<HI, NS>;
       uint32_t a_cnt = 0, items = 0, u = 0;
       // descriptors built once; a stage or sub-tile only adds its offset >> 4
       const uint64_t adesc0 = make_sdesc(smem_u32(sA), 16, L::kSBO, L::kSwizzleLayout);
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(EpiCfg<HI>::THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    using E = EpiCfg<HI>;
+    using E = EpiCfg<HI, NS>;
     const int ew = warp - 2;             // 0 .. 4 * NGRP - 1
     const int grp = ew >> 2;             // drains groups u with u % NGRP == grp
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
@@ -619,7 +622,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
   p.q_begin = a.q_begin;
   p.q_count = a.q_count;
   p.nb = (a.q_count + QPS - 1) / QPS;
-  if (p.nb > kMaxNB) p.nb = kMaxNB;
+  if (p.nb > L::kMaxNB) p.nb = L::kMaxNB;
   const int per_group = p.nb * QPS;
   p.groups_per_seq = (a.q_count + per_group - 1) / per_group;
   p.wait_ns = c.wait_ns;
@@ -636,16 +639,18 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
     }
     return n * a.B;
   };
+  // CTA slots of the grid (the one-query form runs two CTAs per SM)
+  const int slots = EpiCfg<HI, NS>::CTAS_PER_SM * c.num_sms;
   p.kc = kKC;
   long long items = count_items(p.kc);
-  if (items < 4LL * c.num_sms) {
+  if (items < 4LL * slots) {
     // few items (decode: one query group per sequence): the key-run length
     // that gives the busiest CTA the fewest key tiles, then the fewest items
     // (each item reloads its queries and weights)
     long long best = -1;
     for (int kc = kKC; kc >= 4; --kc) {
       const long long n = count_items(kc);
-      const long long load = (n + c.num_sms - 1) / c.num_sms * kc;
+      const long long load = (n + slots - 1) / slots * kc;
       if (best < 0 || load < best) {
         best = load;
         p.kc = kc;
@@ -653,7 +658,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
       }
     }
   }
-  const int grid = (int)(items < c.num_sms ? items : c.num_sms);
+  const int grid = (int)(items < slots ? items : slots);
   if (grid <= 0) return cudaSuccess;
   // the contiguous fast paths (no lengths, no paging, stride 1, no repair
   // list), with score rows or candidate lists as the output
@@ -664,7 +669,7 @@ cudaError_t launch_tc(const LaunchCtx& c, const IndexerArgs& a) {
                             : indexer_tc_kernel<DI, HI, false, false, NS>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  kern<<<grid, EpiCfg<HI>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
+  kern<<<grid, EpiCfg<HI, NS>::THREADS, L::kAlloc, c.stream>>>(tm_k, tm_q, p);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -676,15 +681,19 @@ cudaError_t launch_di(const LaunchCtx& c, const IndexerArgs& a) {
     case 8: return launch_tc<DI, 8, kNSub>(c, a);
     case 16: return launch_tc<DI, 16, kNSub>(c, a);
     case 32: return launch_tc<DI, 32, kNSub>(c, a);
-    // one query per sequence (decode): sub-tiles of one query's 64 heads
-    case 64: return a.q_count == 1 ? launch_tc<DI, 64, 64>(c, a) : launch_tc<DI, 64, kNSub>(c, a);
+    // one query per sequence (decode, scores out): sub-tiles of one query's
+    // 64 heads, two CTAs per SM
+    case 64:
+      return a.q_count == 1 && a.thr == nullptr ? launch_tc<DI, 64, 64>(c, a) : launch_tc<DI, 64, kNSub>(c, a);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-int indexer_epilogue_warps(int H_I) { return (H_I >= 32 ? EpiCfg<64>::EPI_THREADS : EpiCfg<4>::EPI_THREADS) / 32; }
+int indexer_epilogue_warps(int H_I) {
+  return (H_I >= 32 ? EpiCfg<64, kNSub>::EPI_THREADS : EpiCfg<4, kNSub>::EPI_THREADS) / 32;
+}
 
 cudaError_t launch_indexer(const LaunchCtx& c, const IndexerArgs& a) {
   if (a.q_count <= 0 || a.B <= 0) return cudaSuccess;
