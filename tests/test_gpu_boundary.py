@@ -295,3 +295,27 @@ def test_prefill_in_query_blocks_equals_one_call():
     # summation order, LSE to 1e-4
     assert torch.allclose(got.out.float(), ref.out.float(), atol=2e-2, rtol=2e-2)
     assert torch.allclose(got.lse, ref.lse, atol=1e-4, rtol=1e-5)
+
+
+def test_indexer_single_query_launch_equals_full_launch():
+    """dsa_indexer_scores for one query row of a prefill (the one-query form:
+    N = 64 sub-tiles, two CTAs per SM) gives that row's scores bit for bit as
+    a launch over all rows does (the same FP8 products, K order and head
+    order), on every visible key."""
+    wl = Workload("one_row", B=2, T=40, S=5000, H_I=64, D_I=128, H=8, d_k=80, d_v=64, k=256, q_block=40, seed=47)
+    inp = make_inputs(wl, "cuda")
+    inp.pop("needle_pos", None)
+    shape = dsa.make_shape(wl)
+    ld = (wl.S + 63) // 64 * 64
+    full = torch.full((wl.B * wl.T, ld), float("nan"), device="cuda")
+    dsa.indexer_scores(shape, inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], 0, wl.T, full)
+    for t in (0, 17, wl.T - 1):
+        one = torch.full((wl.B, ld), float("nan"), device="cuda")
+        dsa.indexer_scores(shape, inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], t, 1, one)
+        st, det = dsa.device_error()
+        assert st == 0, (st, hex(det))
+        n = wl.S - wl.T + t + 1
+        for b in range(wl.B):
+            a = one[b, :n].cpu().numpy()
+            r = full[b * wl.T + t, :n].cpu().numpy()
+            assert np.array_equal(a, r), (t, b, np.max(np.abs(a - r)))

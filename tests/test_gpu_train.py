@@ -175,3 +175,52 @@ def test_indexer_backward_shapes(name, B, T, S, H_I, k, page, ragged):
         else:
             got = dk_np[b]
         _close(got, dk_ref, 2e-5, f"dk b={b}")
+
+
+@pytest.mark.parametrize("sparse", [False, True], ids=["dense", "sparse"])
+def test_kl_target_paged_ragged(sparse):
+    """dsa_kl_target over page pools (page 64, random order) with ragged
+    lengths, against the oracle's target rows; the dense stage reads every
+    visible key, the sparse one a random set with empty slots anywhere.  The
+    lse fed in is the oracle's own (natural log over the same keys), so only
+    the target's arithmetic is under test: 1e-5 absolute (entries are
+    probabilities)."""
+    wl = Workload("kl_paged", B=2, T=6, S=900, H_I=8, D_I=64, H=128, d_k=576, d_v=512, k=200, q_block=6, seed=95)
+    inp = make_inputs(wl, "cuda")
+    inp.pop("needle_pos", None)
+    lengths = [wl.S, wl.S - 123]
+    sl = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    pin, table, num_pages = to_paged(inp, wl, 64, 96)
+    shape = dsa.make_shape(wl, seqlens=sl, block_table=table, page_size=64, num_pages=num_pages)
+    rng = np.random.default_rng(97)
+    tau = float(O.default_tau(wl.d_k))
+    sel = None
+    if sparse:
+        sel = np.full((wl.B, wl.T, wl.k), -1, np.int32)
+        for b in range(wl.B):
+            for t in range(wl.T):
+                n = lengths[b] - wl.T + t + 1
+                keys = rng.choice(n, size=min(wl.k, n) - 7, replace=False)
+                sel[b, t, rng.permutation(wl.k)[: keys.size]] = keys
+    lse = np.zeros((wl.B, wl.T, wl.H), np.float32)
+    refs = {}
+    for b in range(wl.B):
+        d = O.from_inputs({k_: v.cpu() for k_, v in inp.items()}, b)
+        for t in range(wl.T):
+            pos = lengths[b] - wl.T + t
+            keys = np.arange(pos + 1) if sel is None else np.unique(sel[b, t][sel[b, t] >= 0])
+            z = tau * (d["q"][t] @ d["kv"][keys].T)
+            m = z.max(axis=1)
+            lse[b, t] = m + np.log(np.exp(z - m[:, None]).sum(axis=1))
+            refs[(b, t)] = O.kl_target_row(d["q"][t], d["kv"], pos, tau, None if sel is None else sel[b, t])
+    ld = (wl.S + 63) // 64 * 64
+    target = torch.zeros(wl.B * wl.T, ld, device="cuda")
+    idx = None if sel is None else torch.from_numpy(sel).cuda()
+    dsa.kl_target(shape, pin["q"], pin["kv"], torch.from_numpy(lse).cuda(), 0, wl.T, target, idx)
+    st, det = dsa.device_error()
+    assert st == 0, (st, hex(det))
+    tg = target.cpu().numpy()
+    for (b, t), p in refs.items():
+        pos = lengths[b] - wl.T + t
+        keys = np.arange(pos + 1) if sel is None else np.unique(sel[b, t][sel[b, t] >= 0])
+        assert np.max(np.abs(tg[b * wl.T + t, keys] - p[keys])) < 1e-5, (b, t)
