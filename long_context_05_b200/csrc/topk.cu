@@ -85,7 +85,8 @@ __device__ __forceinline__ unsigned int block_scan(unsigned int v, unsigned int*
 }
 
 // Find the bin holding the rank-th largest key (rank >= 1) among bins
-// counted in hist[0..nb) (nb = kBins or 256; larger bin = larger keys).
+// counted in hist[0..nb) (nb a power of two up to kBins; larger bin = larger
+// keys).
 // Returns the bin in *bin and the count of keys in higher bins in *above.
 __device__ void find_bin(const unsigned int* hist, int nb, unsigned int rank, unsigned int* warp_tot,
                          unsigned int* s_bin, unsigned int* s_above, unsigned int* s_total) {
@@ -118,26 +119,29 @@ __device__ void find_bin(const unsigned int* hist, int nb, unsigned int rank, un
 
 // Radix select over `count` keys delivered by key_of(i) that all share the bits
 // in `mask` with `prefix`: finds the rank-th largest key (rank >= 1), refining
-// 8 bits at a time from bit `hi` down to bit 0.  Returns the key; *krem gets
-// how many keys equal to it belong to the top `rank`.
+// 11 bits at a time (the kBins histogram) from bit `hi` down to bit 0.
+// Returns the key; *krem gets how many keys equal to it belong to the top
+// `rank`.
 template <class KeyOf>
 __device__ unsigned int radix_select(KeyOf key_of, int count, unsigned int prefix, unsigned int mask, int hi,
                                      unsigned int rank, unsigned int* hist, unsigned int* warp_tot,
                                      unsigned int* s_bin, unsigned int* s_above, unsigned int* s_total,
                                      unsigned int* krem_out) {
+  constexpr int kDigit = 11;                  // kBins = 2^11
   unsigned int krem = rank;
   while (hi > 0) {
-    const int bits = hi >= 8 ? 8 : hi;
+    const int bits = hi >= kDigit ? kDigit : hi;
     const int shift = hi - bits;
     const unsigned int dmask = (1u << bits) - 1u;
-    for (int x = threadIdx.x; x < 256; x += kThreads) hist[x] = 0u;
+    const int nb = 1 << bits;
+    for (int x = threadIdx.x; x < nb; x += kThreads) hist[x] = 0u;
     __syncthreads();
     for (int i = threadIdx.x; i < count; i += kThreads) {
       const unsigned int key = key_of(i);
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
     }
     __syncthreads();
-    find_bin(hist, 256, krem, warp_tot, s_bin, s_above, s_total);
+    find_bin(hist, nb, krem, warp_tot, s_bin, s_above, s_total);
     prefix |= *s_bin << shift;
     mask |= dmask << shift;
     krem -= *s_above;
