@@ -359,19 +359,22 @@ __device__ void histogram_pass(const float* row, int lo, int hi, unsigned int* h
 
 // One pass over the row when a lower bound on the k-th key is known: every
 // key at or above `lo` becomes a candidate.  Rows of at most kCap keys take
-// all keys; longer rows estimate the bound from a sample (four adjacent keys
-// out of every 64 x step, about 1.5 k / (16 step) + 16 sampled keys above
-// it, so about 1.5 k keys of the row are expected above it).  Returns false
+// all keys; longer rows estimate the bound from a sample of at most
+// kSampleBlocks groups of four adjacent keys, one out of every 64 x step keys:
+// the bound has about 1.5 k / (16 step) + 16 sampled keys above it, so about
+// 1.5 k + 256 step keys of the row are expected above it (3.3 k at 32K keys,
+// 4.1 k at 128K; k is short of it with negligible probability).  Returns false
 // (nothing written) when the candidates are fewer than k or do not fit in
 // shared memory; the caller then runs the two-pass histogram path.
+constexpr int kSampleBlocks = 512;
 __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& sm, DevErr* err) {
   const int tid = threadIdx.x;
   const float4* r4 = reinterpret_cast<const float4*>(row);
   unsigned int lo = 0u;
   if (n > kCap) {
     const int nblk = n / 64;                         // 64-key blocks (>= 128 here)
-    const int step = (nblk + kCap / 4 - 1) / (kCap / 4);
-    const int ns = nblk / step;                      // sampled blocks, <= kCap / 4
+    const int step = (nblk + kSampleBlocks - 1) / kSampleBlocks;
+    const int ns = nblk / step;                      // sampled blocks, <= kSampleBlocks
     const int m = 4 * ns;
     const int rs = min(m, (3 * k) / (2 * 16 * step) + 16);
     for (int i = tid; i < ns; i += kThreads) {
