@@ -102,7 +102,7 @@ struct Cfg {
   // one set per S buffer: [kSBuf][2 sides][128 rows]
   static constexpr int OFF_XM = OFF_MASK + SLOTS * 4;
   static constexpr int OFF_BAR = OFF_XM + kSBuf * 2 * 128 * 4;
-  static constexpr int NBARS = 2 + 2 * SLOTS + 3 * kSBuf + 1 + kSBuf * 4 + 4;
+  static constexpr int NBARS = 2 + 2 * SLOTS + 3 * kSBuf + 1 + kSBuf * 4 + 4 + SLOTS;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   // the dynamic shared memory base is checked for 1024-byte alignment at run
@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = pv_done + kSBuf;
   uint64_t* mx_bar = mma_done + 1;             // [kSBuf][4 quarters] both partial maxima written
   uint64_t* lx_bar = mx_bar + kSBuf * 4;       // [4 quarters] both partial row sums written
+  uint64_t* kv_kfree = lx_bar + 4;             // [kSlots] Q K^T of the slot's chunk done (MMA commit)
   float* sXM = reinterpret_cast<float*>(smem + C::OFF_XM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&kv_full[i], 32 * kGatherPerSlot);
       mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_kfree[i], 1);
     }
     for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&s_full[i], 1);
@@ -238,10 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int c16 = lane & 7, rg = lane >> 3;  // 16-byte column chunk, row group
     const int32_t* irow = dense ? nullptr : p.idx + (size_t)row * p.k;
-    // the sequence's rows of a contiguous cache; in the paged form, the cache
-    // row of its key 0 (every sequence has at least T keys), which empty
-    // slots copy (pool row 0 if that page is unmapped)
-    const uint16_t* kvb = p.kv + (size_t)b * p.S * DK;
+    // in the paged form, the cache row of the sequence's key 0 (every
+    // sequence has at least T keys), which empty slots copy (pool row 0 if
+    // that page is unmapped); a contiguous cache copies row b * S
     long long row0 = PAGED && nchunks > 0 ? p.map.row<true>(b, 0) : 0;
     if (row0 < 0) row0 = 0;
     // indices of this half of chunk j, loaded one chunk ahead
@@ -254,13 +255,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     load_idx(0);
+    // The atoms of a key row that this CTA's P V reads (its value half, or
+    // the separate value atoms) are refilled once P V of the slot's last
+    // chunk is done; the others as soon as its Q K^T is, so most of the next
+    // gather overlaps the softmax and P V before it.
+    const int vlo = half * C::DVH / 64, vhi = ((half + 1) * C::DVH - 1) / 64;
+    auto reads_v = [&](int a) { return !SEPV && a >= vlo && a <= vhi; };
     for (int j = 0; j < nchunks; ++j) {
       const int st = 2 * (j % C::NCH) + h;     // ring slot of this half of chunk j
       int iv[kSlotKeys / 4];
 #pragma unroll
       for (int m = 0; m < kSlotKeys / 4; ++m) iv[m] = ivn[m];
-      if (j >= C::NCH && !wwait(&kv_empty[st], (uint32_t)((j / C::NCH) - 1) & 1)) { fail(1); break; }
+      if (j >= C::NCH && !wwait(&kv_kfree[st], (uint32_t)((j / C::NCH) - 1) & 1)) { fail(1); break; }
       uint8_t* slotp = sKV + st * C::SLOT_ATOM;
+      size_t crows[kSlotKeys / 4];
       uint32_t mask = 0;
 #pragma unroll
       for (int m = 0; m < kSlotKeys / 4; ++m) {
@@ -289,14 +297,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         // finite row of the caller's cache), which then meets probability 0
         // in P V
         const size_t crow = PAGED ? (size_t)(valid ? cr : row0) : (size_t)b * p.S + (valid ? v : 0);
-        const uint16_t* src = PAGED ? p.kv + crow * DK : kvb + (size_t)(valid ? v : 0) * DK;
+        crows[m] = crow;
+        // phase 1: key atoms that P V does not read
+        const uint16_t* src = p.kv + crow * DK;
 #pragma unroll
         for (int a0 = 0; a0 < C::NATOM; a0 += kGatherPerSlot) {
           const int a = a0 + g;
-          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2)
+          if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2 && !reads_v(a))
             cp_async16(slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
         }
-        if constexpr (SEPV) {
+      }
+      // phase 2: the atoms P V reads, once P V of the slot's last chunk is done
+      if (j >= C::NCH && !wwait(&kv_empty[st], (uint32_t)((j / C::NCH) - 1) & 1)) { fail(1); break; }
+#pragma unroll
+      for (int m = 0; m < kSlotKeys / 4; ++m) {
+        const int r = rg + 4 * m;
+        const size_t crow = crows[m];
+        if constexpr (!SEPV) {
+          const uint16_t* src = p.kv + crow * DK;
+#pragma unroll
+          for (int a0 = 0; a0 < C::NATOM; a0 += kGatherPerSlot) {
+            const int a = a0 + g;
+            if (a < C::NATOM && a * 128 + c16 * 16 < DK * 2 && reads_v(a))
+              cp_async16(slotp + a * C::ATOM_STRIDE + r * 128 + ((c16 ^ (r & 7)) << 4), src + a * 64 + c16 * 8);
+          }
+        } else {
           // this CTA's value columns [half * DVH, (half + 1) * DVH) of the
           // value row, in atoms NATOM, NATOM + 1, ...
           const uint16_t* vsrc = p.v + crow * DV + half * C::DVH;
@@ -395,6 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             mma_commit(&s_full[sb]);
+            // the slots' atoms that P V does not read may be refilled now
+            mma_commit(&kv_kfree[s0]);
+            mma_commit(&kv_kfree[s0 + 1]);
             ++qk;
             progressed = true;
           }
@@ -429,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // by their consumers; make sure they have landed before the CTA exits
       for (int c = max(0, 2 * pv - kSlots); c < 2 * pv; ++c)
         mbar_wait(&kv_empty[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
+      for (int c = max(0, 2 * qk - kSlots); c < 2 * qk; ++c)
+        mbar_wait(&kv_kfree[c % kSlots], (c / kSlots) & 1, p.wait_ns, no_abort);
       for (int i = max(0, pv - kSBuf); i < pv; ++i)
         mbar_wait(&pv_done[i % kSBuf], (i / kSBuf) & 1, p.wait_ns, no_abort);
       for (int i = max(0, qk - kSBuf); i < qk; ++i)
