@@ -65,11 +65,11 @@ DECODE = "decode_128k_b8"
 # for the kernel source it was taken from, so the bench reports it only while
 # that source's hash matches.
 ATTN_TRAFFIC = {"workload": "prefill_128k", "kernel": "sparse_attn",
-                # DRAM read + write of one prefill_chunk_128k launch (92.37 MB +
-                # 32.00 MB, ncu) times 256, the ratio of query rows
-                "bytes": 92.37e6 * 256 + 32.00e6 * 256,
+                # DRAM read + write of one prefill_chunk_128k launch (92.39 MB +
+                # 30.67 MB, ncu) times 256, the ratio of query rows
+                "bytes": 92.39e6 * 256 + 30.67e6 * 256,
                 "source": "long_context_05_b200/csrc/sparse_attn.cu",
-                "sha256": "1014d28eb4e008b7b4ad86ac641c8086294879e2df7ff9a8abf6871d01a86f78"}
+                "sha256": "7606374af7813d86460dc014ed6b075e2dd843c8d1b6348b974638678cc1c406"}
 
 
 def measured_traffic(workload: str, kernel: str):
