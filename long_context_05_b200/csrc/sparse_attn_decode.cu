@@ -475,23 +475,36 @@ __global__ void __launch_bounds__(256) attn_combine_f16_kernel(const __half* par
   const float* ls = part_lse + (size_t)row * nsplit * H + h;
   const __half* po = part_o + ((size_t)row * nsplit * H + h) * DV + d0;   // split s at + s * H * DV
   float mx = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, ls[(size_t)s * H]);
+  if (nsplit > kBatch)
+    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, ls[(size_t)s * H]);
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   float wsum = 0.f;
-  if (mx != -INFINITY) {
-    for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
-      float w[kBatch];
-      uint4 v[kBatch];
+  for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
+    // every load of the batch is issued at once (one memory latency): an
+    // empty split's partial was never written, so its value is read and
+    // then replaced by zero rather than fetched only when its lse is finite
+    float l[kBatch];
+    uint4 v[kBatch];
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int s = s0 + i;
-        const float l = s < nsplit ? ls[(size_t)s * H] : -INFINITY;
-        w[i] = l == -INFINITY ? 0.f : exp2f(l - mx);
-        v[i] = l == -INFINITY ? make_uint4(0u, 0u, 0u, 0u)
-                              : *reinterpret_cast<const uint4*>(po + (size_t)s * H * DV);
-      }
+    for (int i = 0; i < kBatch; ++i) {
+      const int s = s0 + i;
+      l[i] = s < nsplit ? ls[(size_t)s * H] : -INFINITY;
+      v[i] = s < nsplit ? *reinterpret_cast<const uint4*>(po + (size_t)s * H * DV) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (nsplit <= kBatch) {
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) mx = fmaxf(mx, l[i]);
+    }
+    if (mx == -INFINITY) break;
+    float w[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      w[i] = l[i] == -INFINITY ? 0.f : exp2f(l[i] - mx);
+      if (l[i] == -INFINITY) v[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    {
 #pragma unroll
       for (int i = 0; i < kBatch; ++i) {
         wsum += w[i];
