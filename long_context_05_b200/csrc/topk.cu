@@ -49,9 +49,9 @@ constexpr int kCap = 8192;            // candidates held in shared memory
 constexpr int kSegBlocks = 16;        // blocks per row in the split (decode) path
 // Split-path workspace per row, in 32-bit words: histogram | counters (keys
 // written, candidates) | candidate keys | candidate indices.
-constexpr int kWsHist = 0;
-constexpr int kWsCtr = kBins;
-constexpr int kWsKeys = kBins + 4;
+constexpr int kWsHist = 0;                     // kSegBlocks segment histograms of kBins words
+constexpr int kWsCtr = kSegBlocks * kBins;     // written, candidates, segments done, (spare)
+constexpr int kWsKeys = kWsCtr + 4;
 constexpr int kWsIdx = kWsKeys + kCap;
 constexpr int kWsRowWords = kWsIdx + kCap;
 
@@ -623,8 +623,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---------------------------------------------------------------- split path
-// Workspace per row: hist[kBins] u32.  Kernel 1 adds each segment's histogram;
-// kernel 2 (one block per row) finds the bin and runs steps 2-3.
+// The allocation-free form (dsa_topk_static): a histogram array of kBins
+// words per row, cleared by topk_zero_kernel; topk_seg_hist_kernel adds each
+// segment's histogram, topk_seg_select_kernel (one block per row) finds the
+// bin and runs steps 2-3.
 
 __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, unsigned int* ghist, int hstride, DevErr* err) {
   __shared__ unsigned int hist[kBins];
@@ -647,131 +649,157 @@ __global__ void __launch_bounds__(kThreads, 1) topk_seg_hist_kernel(TopkArgs a, 
     if (hist[x]) atomicAdd(&gh[x], hist[x]);
 }
 
-// Split path, step 2 over one segment of a row: find bin B from the row's
-// histogram, write the keys above B, append bin B's keys to the candidates.
-__global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
+// Split path (few long rows, as in decode), two launches:
+//  1. topk_seg_hist2_kernel: each of kSegBlocks blocks of a row writes the
+//     histogram of its segment into the row's slot for it (plain stores, so
+//     nothing needs clearing first); segment 0 also clears the row's counters;
+//  2. topk_seg_collect_final_kernel: every block sums the row's segment
+//     histograms, finds the threshold bin B, writes its segment's keys above
+//     B and appends bin B's keys to the row's candidates; the last block of
+//     the row to finish (an atomic count, no waiting) then selects the rest
+//     from the candidates.
+
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_hist2_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
   __shared__ unsigned int hist[kBins];
   pdl_launch_dependents();
   pdl_wait();
-  __shared__ unsigned int warp_tot[kWarps];
-  __shared__ unsigned int s_bin, s_above, s_total;
+  const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
+  int b, t, n;
+  const float* row;
+  int32_t* out;
+  row_setup(a, r, err, &b, &t, &n, &row, &out);
+  if (n <= a.k) return;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) hist[x] = 0u;
+  __syncthreads();
+  const int per = ((n + kSegBlocks - 1) / kSegBlocks + 3) & ~3;
+  const int lo = seg * per, hi = min(n, lo + per);
+  if (lo < hi) histogram_pass(row, lo, hi, hist);
+  __syncthreads();
+  unsigned int* w = ws + (size_t)r * kWsRowWords;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) w[kWsHist + seg * kBins + x] = hist[x];
+  if (seg == 0 && threadIdx.x < 4) w[kWsCtr + threadIdx.x] = 0u;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_seg_collect_final_kernel(TopkArgs a, unsigned int* ws,
+                                                                            DevErr* err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  // the decode attention may start its prologue now
+  pdl_launch_dependents();
+  pdl_wait();
+  unsigned int* hist = sm.hist;
+  unsigned int* warp_tot = sm.warp_tot;
   const int r = blockIdx.x / kSegBlocks, seg = blockIdx.x - r * kSegBlocks;
   int b, t, n;
   const float* row;
   int32_t* out;
   row_setup(a, r, err, &b, &t, &n, &row, &out);
   const int k = a.k;
-  if (n <= k) return;
+  if (n <= k) {
+    if (seg == 0)
+      for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
+    return;
+  }
   unsigned int* w = ws + (size_t)r * kWsRowWords;
-  for (int x = threadIdx.x; x < kBins; x += kThreads) hist[x] = w[kWsHist + x];
-  if (threadIdx.x == 0) s_bin = 0xFFFFFFFFu;
+  // the row's histogram: the sum of its segments' (all loads in flight)
+  for (int x = threadIdx.x; x < kBins; x += kThreads) {
+    unsigned int v[kSegBlocks];
+#pragma unroll
+    for (int sg = 0; sg < kSegBlocks; ++sg) v[sg] = w[kWsHist + sg * kBins + x];
+    unsigned int sum = 0u;
+#pragma unroll
+    for (int sg = 0; sg < kSegBlocks; ++sg) sum += v[sg];
+    hist[x] = sum;
+  }
+  if (threadIdx.x == 0) sm.bin = 0xFFFFFFFFu;
   __syncthreads();
-  find_bin(hist, kBins, (unsigned int)k, warp_tot, &s_bin, &s_above, &s_total);
-  const unsigned int B = s_bin;
-  if (B >= (unsigned)kBins) return;  // reported by the final kernel
+  find_bin(hist, kBins, (unsigned int)k, warp_tot, &sm.bin, &sm.above, &sm.total);
+  const unsigned int B = sm.bin, above = sm.above;
   unsigned int* cnt = w + kWsCtr;
   unsigned int* ncand = w + kWsCtr + 1;
   unsigned int* ck = w + kWsKeys;
   int* ci = reinterpret_cast<int*>(w + kWsIdx);
   const int per = ((n + kSegBlocks - 1) / kSegBlocks + 3) & ~3;
   const int lo = seg * per, hi = min(n, lo + per);
-  if (lo >= hi) return;  // past the end of a short row
-  // Rounds of eight keys per thread (two 16-byte loads), the same number for
-  // every thread: each round counts its hits per thread, one block scan gives
-  // every thread its offsets, and one global atomic per list reserves the
-  // block's range.
-  __shared__ unsigned int s_base_out, s_base_cand;
-  const float4* r4 = reinterpret_cast<const float4*>(row);
-  const int n4lo = lo / 4, n4hi = hi / 4;  // lo is a multiple of 4
-  const int tail = hi - 4 * n4hi;          // fewer than 4 keys after the last 16-byte load
-  const int rounds = (n4hi - n4lo + 2 * kThreads - 1) / (2 * kThreads) + (tail > 0 ? 1 : 0);
-  for (int rd = 0; rd < rounds; ++rd) {
-    float f[8];
-    int x[8];
-    bool ok[8];
-    const int base = n4lo + rd * 2 * kThreads;
-    if (base < n4hi) {
+  __shared__ unsigned int s_base_out, s_base_cand, s_last;
+  if (B < (unsigned)kBins && lo < hi) {
+    // Rounds of eight keys per thread (two 16-byte loads), the same number for
+    // every thread: each round counts its hits per thread, one block scan gives
+    // every thread its offsets, and one global atomic per list reserves the
+    // block's range.
+    const float4* r4 = reinterpret_cast<const float4*>(row);
+    const int n4lo = lo / 4, n4hi = hi / 4;  // lo is a multiple of 4
+    const int tail = hi - 4 * n4hi;          // fewer than 4 keys after the last 16-byte load
+    const int rounds = (n4hi - n4lo + 2 * kThreads - 1) / (2 * kThreads) + (tail > 0 ? 1 : 0);
+    for (int rd = 0; rd < rounds; ++rd) {
+      float f[8];
+      int x[8];
+      bool ok[8];
+      const int base = n4lo + rd * 2 * kThreads;
+      if (base < n4hi) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int i4 = base + u * kThreads + (int)threadIdx.x;
-        const bool v = i4 < n4hi;
-        const float4 q = v ? r4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
-        f[4 * u] = q.x; f[4 * u + 1] = q.y; f[4 * u + 2] = q.z; f[4 * u + 3] = q.w;
+        for (int u = 0; u < 2; ++u) {
+          const int i4 = base + u * kThreads + (int)threadIdx.x;
+          const bool v = i4 < n4hi;
+          const float4 q = v ? r4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          f[4 * u] = q.x; f[4 * u + 1] = q.y; f[4 * u + 2] = q.z; f[4 * u + 3] = q.w;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[4 * u + e] = 4 * i4 + e;
-          ok[4 * u + e] = v;
+          for (int e = 0; e < 4; ++e) {
+            x[4 * u + e] = 4 * i4 + e;
+            ok[4 * u + e] = v;
+          }
+        }
+      } else {  // the last round takes the tail keys, one per thread
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ok[e] = e == 0 && (int)threadIdx.x < tail;
+          x[e] = 4 * n4hi + (int)threadIdx.x;
+          f[e] = ok[e] ? row[x[e]] : 0.f;
         }
       }
-    } else {  // the last round takes the tail keys, one per thread
+      unsigned int up = 0, cb = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        ok[e] = e == 0 && (int)threadIdx.x < tail;
-        x[e] = 4 * n4hi + (int)threadIdx.x;
-        f[e] = ok[e] ? row[x[e]] : 0.f;
+        const unsigned int bin = order_key(f[e]) >> kBinShift;
+        up += (ok[e] && bin > B) ? 1u : 0u;
+        cb += (ok[e] && bin == B) ? 1u : 0u;
       }
-    }
-    unsigned int up = 0, cb = 0;
+      // both counts fit 16 bits: at most 8 per thread and 8192 per block
+      const unsigned int packed = up | (cb << 16);
+      const unsigned int incl = block_scan(packed, warp_tot, &sm.total);
+      const unsigned int excl = incl - packed;
+      if (threadIdx.x == 0) {
+        const unsigned int tot = sm.total;
+        s_base_out = (tot & 0xFFFFu) ? atomicAdd(cnt, tot & 0xFFFFu) : 0u;
+        s_base_cand = (tot >> 16) ? atomicAdd(ncand, tot >> 16) : 0u;
+      }
+      __syncthreads();
+      unsigned int po = s_base_out + (excl & 0xFFFFu), pc = s_base_cand + (excl >> 16);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const unsigned int bin = order_key(f[e]) >> kBinShift;
-      up += (ok[e] && bin > B) ? 1u : 0u;
-      cb += (ok[e] && bin == B) ? 1u : 0u;
-    }
-    // both counts fit 16 bits: at most 8 per thread and 8192 per block
-    const unsigned int packed = up | (cb << 16);
-    const unsigned int incl = block_scan(packed, warp_tot, &s_total);
-    const unsigned int excl = incl - packed;
-    if (threadIdx.x == 0) {
-      const unsigned int tot = s_total;
-      s_base_out = (tot & 0xFFFFu) ? atomicAdd(cnt, tot & 0xFFFFu) : 0u;
-      s_base_cand = (tot >> 16) ? atomicAdd(ncand, tot >> 16) : 0u;
-    }
-    __syncthreads();
-    unsigned int po = s_base_out + (excl & 0xFFFFu), pc = s_base_cand + (excl >> 16);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const unsigned int key = order_key(f[e]);
-      const unsigned int bin = key >> kBinShift;
-      if (ok[e] && bin > B) put(out, k, (int)po++, x[e], err, 10);
-      if (ok[e] && bin == B) {
-        if (pc < (unsigned)kCap) {
-          ck[pc] = key;
-          ci[pc] = x[e];
+      for (int e = 0; e < 8; ++e) {
+        const unsigned int key = order_key(f[e]);
+        const unsigned int bin = key >> kBinShift;
+        if (ok[e] && bin > B) put(out, k, (int)po++, x[e], err, 10);
+        if (ok[e] && bin == B) {
+          if (pc < (unsigned)kCap) {
+            ck[pc] = key;
+            ci[pc] = x[e];
+          }
+          ++pc;
         }
-        ++pc;
       }
+      __syncthreads();  // s_base_* are rewritten by the next round
     }
-    __syncthreads();  // s_base_* are rewritten by the next round
   }
-}
-
-// Split path, step 3: one block per row selects from the collected
-// candidates; more candidates than shared memory holds falls back to the
-// passes over the row.
-__global__ void __launch_bounds__(kThreads, 2) topk_seg_final_kernel(TopkArgs a, unsigned int* ws, DevErr* err) {
-  extern __shared__ uint8_t smem_raw[];
-  // the decode attention may start its prologue now on the idle SMs
-  pdl_launch_dependents();
-  pdl_wait();
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  int b, t, n;
-  const float* row;
-  int32_t* out;
-  row_setup(a, blockIdx.x, err, &b, &t, &n, &row, &out);
-  const int k = a.k;
-  if (n <= k) {
-    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = x < n ? x : -1;
-    return;
-  }
-  const unsigned int* w = ws + (size_t)blockIdx.x * kWsRowWords;
-  for (int x = threadIdx.x; x < kBins; x += kThreads) sm.hist[x] = w[kWsHist + x];
-  if (threadIdx.x == 0) sm.bin = 0xFFFFFFFFu;
+  // the last block of the row to get here finishes the row
+  __threadfence();
   __syncthreads();
-  find_bin(sm.hist, kBins, (unsigned int)k, sm.warp_tot, &sm.bin, &sm.above, &sm.total);
-  const unsigned int B = sm.bin, above = sm.above;
-  const unsigned int inbin = B < (unsigned)kBins ? sm.hist[B] : 0u;
-  const unsigned int written = w[kWsCtr], nc = w[kWsCtr + 1];
+  if (threadIdx.x == 0) s_last = atomicAdd(&w[kWsCtr + 2], 1u) == (unsigned int)(kSegBlocks - 1) ? 1u : 0u;
+  __syncthreads();
+  if (s_last == 0u) return;
+  __threadfence();
+  const unsigned int inbin = B < (unsigned)kBins ? hist[B] : 0u;
+  const unsigned int written = atomicAdd(cnt, 0u), nc = atomicAdd(ncand, 0u);
   __syncthreads();
   if (B >= (unsigned)kBins || written != above || nc != inbin || nc > (unsigned)kCap) {
     // (the first two cannot happen with a consistent histogram; the passes
@@ -780,8 +808,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_seg_final_kernel(TopkArgs a,
     return;
   }
   for (int i = threadIdx.x; i < (int)nc; i += kThreads) {
-    sm.ck[i] = w[kWsKeys + i];
-    sm.ci[i] = static_cast<int>(w[kWsIdx + i]);
+    sm.ck[i] = ck[i];
+    sm.ci[i] = ci[i];
   }
   if (threadIdx.x == 0) sm.cnt = (int)above;
   __syncthreads();
@@ -907,23 +935,18 @@ cudaError_t launch_topk(const LaunchCtx& c, const TopkArgs& a, void* ws, size_t 
     note_launches(1);
     return cudaGetLastError();
   }
-  // four launches, each a programmatic dependent of the one before (the
+  // two launches, each a programmatic dependent of the one before (the
   // first of the indexer's): each starts while its predecessor drains
   unsigned int* w = static_cast<unsigned int*>(ws);
-  e = cudaFuncSetAttribute(topk_seg_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(topk_seg_collect_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  if ((e = launch_pdl(topk_zero_kernel, dim3(64), dim3(256), 0, c.stream, w, rows, (int)kWsRowWords,
-                      (int)kWsKeys)) != cudaSuccess)
-    return e;
-  if ((e = launch_pdl(topk_seg_hist_kernel, dim3(rows * kSegBlocks), dim3(kThreads), 0, c.stream, a, w,
-                      (int)kWsRowWords, c.err)) != cudaSuccess)
-    return e;
-  if ((e = launch_pdl(topk_seg_collect_kernel, dim3(rows * kSegBlocks), dim3(kThreads), 0, c.stream, a, w, c.err)) !=
+  if ((e = launch_pdl(topk_seg_hist2_kernel, dim3(rows * kSegBlocks), dim3(kThreads), 0, c.stream, a, w, c.err)) !=
       cudaSuccess)
     return e;
-  if ((e = launch_pdl(topk_seg_final_kernel, dim3(rows), dim3(kThreads), smem, c.stream, a, w, c.err)) != cudaSuccess)
+  if ((e = launch_pdl(topk_seg_collect_final_kernel, dim3(rows * kSegBlocks), dim3(kThreads), smem, c.stream, a, w,
+                      c.err)) != cudaSuccess)
     return e;
-  note_launches(4);
+  note_launches(2);
   return cudaGetLastError();
 }
 
