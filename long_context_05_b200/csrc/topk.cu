@@ -19,19 +19,20 @@
 //   2. a second pass (the row is now in L2) writes every key above bin B to
 //      the output and copies the keys of bin B, with their indices, into
 //      shared memory;
-//   3. radix select over those candidates (8-bit digits) finds the exact k-th
-//      key `thr`; candidates above it are written, and of the candidates equal
-//      to it the lowest indices are kept (a second radix select on the bitwise
-//      complement of the index picks them).
+//   3. radix select over those candidates (11-bit digits) finds the exact
+//      k-th key `thr`; one block scan places the candidates above it, and of
+//      the candidates equal to it the lowest indices are kept (a second radix
+//      select on the bitwise complement of the index picks them when they do
+//      not all fit).
 // If bin B holds more candidates than shared memory takes, steps 2-3 run as
 // radix passes over the row itself and a final pass in index order.
-// Decode rows (few, long) are split over several blocks for steps 1-2: the
-// blocks of a row add their histograms in the caller's workspace, then each
-// block finds bin B from the row's histogram and, over its own segment,
-// writes the keys above B to the output and appends bin B's keys to a
-// per-row candidate list in the workspace (a block scan of the per-thread
-// counts, then one global atomic per list and block); one block per row
-// finishes step 3 on that list.
+// Decode rows (few, long) are split over several blocks for steps 1-2: each
+// block of a row writes the histogram of its segment into the caller's
+// workspace, then each block sums the row's segment histograms, finds bin B
+// and, over its own segment, writes the keys above B to the output and
+// appends bin B's keys to a per-row candidate list in the workspace (a block
+// scan of the per-thread counts, then one global atomic per list and block);
+// the row's last block to finish runs step 3 on that list.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -186,22 +187,33 @@ __device__ void select_candidates(int nc, unsigned int prefix, unsigned int mask
   unsigned int krem;
   const unsigned int thr = radix_select([ck](int i) { return ck[i]; }, nc, prefix, mask, hi, need, sm.hist,
                                         sm.warp_tot, &sm.bin, &sm.above, &sm.total, &krem);
-  // candidates above thr
-  unsigned int eq_local = 0;
+  // One block scan of (above thr, equal to thr) counts places every output:
+  // the keys above thr first, then, when all of them fit, the equal ones.
+  // Both counts fit 16 bits (at most kCap candidates).
+  const unsigned int base = (unsigned int)sm.cnt;
+  unsigned int gt = 0, eq = 0;
   for (int i = tid; i < nc; i += kThreads) {
-    if (sm.ck[i] > thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 2);
-    eq_local += sm.ck[i] == thr;
+    const unsigned int key = sm.ck[i];
+    gt += key > thr ? 1u : 0u;
+    eq += key == thr ? 1u : 0u;
   }
-  block_scan(eq_local, sm.warp_tot, &sm.total);
-  const unsigned int E = sm.total;
-  if (E == krem) {
-    for (int i = tid; i < nc; i += kThreads)
-      if (sm.ck[i] == thr) put(out, k, atomicAdd(&sm.cnt, 1), sm.ci[i], err, 3);
-    return;
+  const unsigned int packed = gt | (eq << 16);
+  const unsigned int excl = block_scan(packed, sm.warp_tot, &sm.total) - packed;
+  const unsigned int G = sm.total & 0xFFFFu, E = sm.total >> 16;
+  const bool all_eq = E == krem;
+  unsigned int pg = base + (excl & 0xFFFFu), pe = base + G + (excl >> 16);
+  for (int i = tid; i < nc; i += kThreads) {
+    const unsigned int key = sm.ck[i];
+    if (key > thr) put(out, k, (int)pg++, sm.ci[i], err, 2);
+    else if (all_eq && key == thr) put(out, k, (int)pe++, sm.ci[i], err, 3);
   }
+  if (all_eq) return;
   // more equal keys than slots: keep the lowest indices.  Gather the equal
   // candidates' indices and select on ~index (lower index = larger key).
-  if (tid == 0) sm.eq_base = 0;
+  if (tid == 0) {
+    sm.cnt = (int)(base + G);
+    sm.eq_base = 0;
+  }
   __syncthreads();
   for (int i = tid; i < nc; i += kThreads)
     if (sm.ck[i] == thr) {
@@ -385,10 +397,14 @@ __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& 
       sm.ck[4 * i + 3] = order_key(v.w);
     }
     __syncthreads();
+    // The bound only has to lie at or below the rs-th sampled key: two 11-bit
+    // digits of the keys' top 22 bits fix it to within 2^10 units of the
+    // order key, which adds a negligible number of candidates.
     const unsigned int* ck = sm.ck;
     unsigned int krem;
-    lo = radix_select([ck](int i) { return ck[i]; }, m, 0u, 0u, 32, (unsigned int)rs, sm.hist, sm.warp_tot, &sm.bin,
-                      &sm.above, &sm.total, &krem);
+    lo = radix_select([ck](int i) { return ck[i] >> 10; }, m, 0u, 0u, 22, (unsigned int)rs, sm.hist, sm.warp_tot,
+                      &sm.bin, &sm.above, &sm.total, &krem)
+         << 10;
   }
   if (tid == 0) {
     sm.cnt = 0;
