@@ -144,6 +144,12 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// Asynchronous prefetch of the global range [p, p + bytes) into L2; p and
+// bytes are multiples of 16.  Nothing waits for it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ TMEM
 
 // Warp-wide: allocate ncols TMEM columns; the base address lands in *dst (smem).

@@ -382,6 +382,19 @@ constexpr int kSampleBlocks = 512;
 __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& sm, DevErr* err) {
   const int tid = threadIdx.x;
   const float4* r4 = reinterpret_cast<const float4*>(row);
+  // The collection pass reads the row in rounds of 2 x kThreads 16-byte
+  // loads; thread 0 keeps an L2 bulk prefetch kPfAhead rounds ahead of them,
+  // starting before the sample, so that the row streams from HBM while the
+  // block has only two loads per thread of its own in flight.
+  constexpr int kRound4 = 2 * kThreads;
+  constexpr int kPfAhead = 2;
+  const int n4 = n / 4;
+  auto prefetch_round = [&](int j) {
+    const int a = j * kRound4;
+    if (a < n4) sm100::prefetch_l2_bulk(r4 + a, (uint32_t)(min(n4 - a, kRound4) * 16));
+  };
+  if (tid == 0 && n > kCap)
+    for (int j = 0; j < kPfAhead; ++j) prefetch_round(j);
   unsigned int lo = 0u;
   if (n > kCap) {
     const int nblk = n / 64;                         // 64-key blocks (>= 128 here)
@@ -422,9 +435,9 @@ __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& 
     }
   };
   {
-    const int n4 = n / 4;
     int x = tid;
     for (; x + kThreads < n4; x += 2 * kThreads) {
+      if (tid == 0) prefetch_round(x / kRound4 + kPfAhead);
       float4 v[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) v[u] = r4[x + u * kThreads];
