@@ -33,6 +33,8 @@
 // appends bin B's keys to a per-row candidate list in the workspace (a block
 // scan of the per-thread counts, then one global atomic per list and block);
 // the row's last block to finish runs step 3 on that list.
+#include <type_traits>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -424,17 +426,24 @@ __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& 
     sm.ncand = 0;
   }
   __syncthreads();
-  auto visit = [&](float f, int x) {
-    const unsigned int key = order_key(f);
-    if (key >= lo) {
-      const int p = atomicAdd(&sm.ncand, 1);
-      if (p < kCap) {
-        sm.ck[p] = key;
-        sm.ci[p] = x;
+  // Candidate test order_key(f) >= lo.  Above the key of +0.0 (a positive
+  // bound, the usual case) it is a signed compare of the raw bits with
+  // lo & 0x7FFFFFFF, one instruction per key: negative floats, -0.0 and
+  // negative NaNs fail it and positive NaNs pass it, as with the keys.  The
+  // key itself is formed only for the candidates.
+  auto collect = [&](auto raw_tag) {
+    constexpr bool kRaw = decltype(raw_tag)::value;
+    const int rlo = (int)(lo & 0x7FFFFFFFu);
+    auto visit = [&](float f, int x) {
+      const bool hit = kRaw ? __float_as_int(f) >= rlo : order_key(f) >= lo;
+      if (hit) {
+        const int p = atomicAdd(&sm.ncand, 1);
+        if (p < kCap) {
+          sm.ck[p] = order_key(f);
+          sm.ci[p] = x;
+        }
       }
-    }
-  };
-  {
+    };
     int x = tid;
     for (; x + kThreads < n4; x += 2 * kThreads) {
       if (tid == 0) prefetch_round(x / kRound4 + kPfAhead);
@@ -458,7 +467,11 @@ __device__ bool single_pass(const float* row, int n, int k, int32_t* out, Smem& 
       visit(v.w, 4 * x + 3);
     }
     for (int e = 4 * n4 + tid; e < n; e += kThreads) visit(row[e], e);
-  }
+  };
+  if (lo > 0x80000000u)
+    collect(std::true_type{});
+  else
+    collect(std::false_type{});
   __syncthreads();
   const int nc = sm.ncand;
   if (nc < k || nc > kCap) return false;
